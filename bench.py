@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--impl ours|reference]
+
+A step is one whole layer forward (route -> permute -> w13/SwiGLU -> w2 ->
+combine) over one batch of synthetic tokens of the workload (default: the
+decode layer T=8, E=128, top_k=8, H=2048, I=768).  Weights stay resident; the L2
+is flushed (a 256 MiB write) before every step, outside the step's CUDA events.
+
+Under torchrun every rank runs its own replica of the workload (its own tokens,
+the same weights): the layer shards by tokens with no data-path collective, so
+scaling is weak and `value` = all ranks' tokens / the slowest rank's time.
+
+Measured on the device with CUDA events:
+  value        tokens/s of moe_forward with inputs resident in HBM
+  roofline     the dominant kernel's algorithmic bytes (or FLOPs) per launch over
+               its mean duration, from a second pass through moe_forward_timed
+               (events between the stages), against MEASURED_PEAKS.json
+  e2e          the same metric with pinned-host x/logits copied in and out copied
+               back inside every step
+  cpu_baseline the fp64 CPU oracle on a bounded sample (rank 0, N = 1 only)
+
+--impl reference times the fp64 CPU oracle itself (the only reference that
+exists for this layer) on the host cores, on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch of the dominant kernel from an ncu capture, keyed by
+# (workload, kernel); None until a capture of the current kernel exists.
+NCU_TRAFFIC = {}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="target CPU time of the cpu_baseline sample")
+    return p.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- stage work model
+
+def stage_work(w, n_touched):
+    """Algorithmic bytes and FLOPs per launch of each stage (not counting padding
+    or re-reads).  n_touched = experts with at least one routed row."""
+    T, E, k, H, I = w.T, w.E, w.k, w.H, w.I
+    R = T * k
+    return {
+        "route_permute": dict(bytes=T * E * 4 + R * (4 + 4) + R * 4 + (E + 1) * 4, flops=0),
+        "w13": dict(bytes=n_touched * 2 * I * H * 2 + T * H * 2 + R * I * 2,
+                    flops=2 * R * 2 * I * H),
+        "w2": dict(bytes=n_touched * H * I * 2 + R * I * 2 + R * H * 2, flops=2 * R * H * I),
+        "combine": dict(bytes=R * H * 2 + R * 4 + T * H * 2, flops=0),
+    }
+
+
+def roofline_entry(stage, work, ms, peaks, peak_kind, sustained, traffic):
+    t = ms / 1e3
+    hbm_t = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    tc_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    tc_t = work["flops"] / (tc_peak * 1e12) if work["flops"] else 0.0
+    if tc_t > hbm_t:
+        achieved = work["flops"] / t / 1e12
+        return {"kernel": stage, "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "traffic": traffic, "algorithmic": work["flops"], "ms": round(ms, 5),
+                "peak_source": f"{peak_kind} ({'sustained' if sustained else 'burst'} bf16)"}
+    achieved = work["bytes"] / t / 1e9
+    return {"kernel": stage, "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "algorithmic": work["bytes"], "ms": round(ms, 5),
+            "peak_source": f"{peak_kind} (copy bandwidth)"}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index, period=0.01):
+        self.period = period
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no clock data rather than guess
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def report(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(w, d_host, seconds):
+    """Time the fp64 oracle on a bounded sample of the workload; returns tokens/s info."""
+    import numpy as np
+
+    import oracle
+
+    T, k, H, I = w.T, w.k, w.H, w.I
+    x, logits, w13, w2 = d_host
+    per_token_macs = k * 3 * H * I
+    full_layer = T * per_token_macs <= 2e9
+    done_tokens = 0
+    calls = 0
+    t0 = time.perf_counter()
+    if full_layer:
+        while True:
+            oracle.forward(x, logits, w13, w2, k)
+            done_tokens += T
+            calls += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        sample = f"whole layer ({T} tokens) x {calls}"
+    else:
+        n = max(1, min(T, int(oracle.num_threads())))
+        ids, _ = oracle.route(logits, k)
+        tok = list(range(n))
+        used = set(ids[tok].reshape(-1).tolist())
+        w13s = [w13[e] if e in used else None for e in range(w.E)]
+        w2s = [w2[e] if e in used else None for e in range(w.E)]
+        while True:
+            oracle.forward_tokens(x, logits, w13s, w2s, k, tok, I)
+            done_tokens += n
+            calls += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        sample = f"{n} of {T} tokens x {calls}"
+    dt = time.perf_counter() - t0
+    return done_tokens / dt, sample, dt
+
+
+def reference_arm(args, rank, world):
+    """Times the fp64 CPU oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from mixture_experts_layer_logits_b200 import workloads as wl
+
+    w = wl.WORKLOADS[args.workload]
+    d = wl.make_inputs(w, seed=args.seed, device="cpu", weights=False)
+    logits = d["logits"].numpy()
+    cfg = dict(w.as_dict())
+    if w.has_ffn:
+        x = wl.bf16_bits(d["x"])
+        # only the experts the sampled tokens select are materialised on the host
+        ids, _ = oracle.route(logits, w.k)
+        n = max(1, min(w.T, oracle.num_threads()))
+        tok = list(range(n))
+        used = sorted(set(ids[tok].reshape(-1).tolist()))
+        w13s = [None] * w.E
+        w2s = [None] * w.E
+        for e in used:
+            a, b = wl.make_expert_weights(w, e, seed=args.seed, device="cpu")
+            w13s[e], w2s[e] = wl.bf16_bits(a), wl.bf16_bits(b)
+
+        def step():
+            oracle.forward_tokens(x, logits, w13s, w2s, w.k, tok, w.I)
+            return n
+        sample = f"{n} of {w.T} tokens per step"
+        metric_unit = "tokens/s"
+    else:
+        def step():
+            ids, _ = oracle.route(logits, w.k)
+            oracle.permute(ids, w.E)
+            return w.T
+        sample = f"all {w.T} tokens per step (route + permute)"
+        metric_unit = "tokens/s"
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    toks = 0
+    for _ in range(args.steps):
+        toks += step()
+    dt = time.perf_counter() - t0
+    value = toks / dt
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": metric_name(w), "value": round(value, 3),
+        "unit": metric_unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": cfg,
+        "cpu_baseline": {"value": round(value, 3), "unit": metric_unit, "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": metric_unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "note": "fp64 CPU oracle of the layer (no other implementation of this layer exists)",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def metric_name(w):
+    return ("MoE layer forward tokens/s at 1 B200 (us/layer in ms_per_step)" if w.has_ffn
+            else "MoE routing (route + permute) tokens/s at 1 B200")
+
+
+# ---------------------------------------------------------------- our arm
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import numpy as np
+    import torch
+
+    import mixture_experts_layer_logits_b200 as moe
+    from mixture_experts_layer_logits_b200 import build as cuda_build
+    from mixture_experts_layer_logits_b200 import workloads as wl
+
+    if rank == 0:
+        cuda_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+        dist.barrier()
+    moe.load_library()
+
+    w = wl.WORKLOADS[args.workload]
+    if not w.has_ffn:
+        raise SystemExit("bench.py times the whole layer; pick a workload with an FFN")
+    T, E, k, H, I = w.T, w.E, w.k, w.H, w.I
+    R = T * k
+    # this rank's tokens; weights are the same on every rank
+    logits = wl.make_logits(w, seed=args.seed + rank, device=dev)
+    x = wl.make_x(w, seed=args.seed + rank, device=dev)
+    w13, w2 = wl.make_weights(w, seed=args.seed, device=dev)
+    ws = moe.workspace(T, E, k, H, I, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    wts = torch.empty(T, k, dtype=torch.float32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    rows = torch.empty(R, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        moe.moe_forward(x, logits, w13, w2, k, ws=ws, out=out, topk_ids=ids, topk_weights=wts,
+                        expert_offsets=off, permuted_rows=rows)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+
+    def max_over_ranks(v):
+        if not pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        fwd()
+    barrier()
+    if moe.moe_device_status(ws) != moe.MOE_OK:
+        raise SystemExit("device error during warm-up")
+    n_touched = int((off[1:] - off[:-1] > 0).sum().item())
+
+    # ---- pass A: the timed steps
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier()
+    with ClockSampler(local) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            fwd()
+            ev[i][1].record(stream)
+        barrier()
+        t_wall = time.perf_counter() - t_wall
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = max_over_ranks(statistics.mean(step_ms))
+    if moe.moe_device_status(ws) != moe.MOE_OK:
+        raise SystemExit("device error during the timed steps")
+
+    # ---- pass B: stage durations through moe_forward_timed
+    KB = min(K, 200)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(KB)]
+    for evs in sev:  # materialise the events (torch creates them on first record)
+        for e in evs:
+            e.record(stream)
+    barrier()
+    for i in range(KB):
+        flush.zero_()
+        moe.moe_forward_timed(x, logits, w13, w2, k, sev[i], ws=ws, out=out, topk_ids=ids,
+                              topk_weights=wts, expert_offsets=off, permuted_rows=rows)
+    barrier()
+    names = ["route_permute", "w13", "w2", "combine"]
+    stage_ms = {n: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(KB))
+                for j, n in enumerate(names)}
+    stage_ms = {n: max_over_ranks(v) for n, v in stage_ms.items()}
+
+    # ---- pass C: end to end from pinned host memory
+    KC = min(K, 200)
+    x_h = x.cpu().pin_memory()
+    logits_h = logits.cpu().pin_memory()
+    out_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(KC)]
+    barrier()
+    for i in range(KC):
+        flush.zero_()
+        eev[i][0].record(stream)
+        x.copy_(x_h, non_blocking=True)
+        logits.copy_(logits_h, non_blocking=True)
+        fwd()
+        out_h.copy_(out, non_blocking=True)
+        eev[i][1].record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in eev))
+    h2d = x_h.numel() * x_h.element_size() + logits_h.numel() * logits_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_kind = load_peaks()
+    work = stage_work(w, n_touched)
+    dominant = max(("w13", "w2", "route_permute", "combine"), key=lambda n: stage_ms[n])
+    sustained = K * ms > 1000.0  # a seconds-long timed region runs at the power-capped clock
+    roof = roofline_entry(dominant, work[dominant], stage_ms[dominant], peaks, peak_kind,
+                          sustained, NCU_TRAFFIC.get((w.name, dominant)))
+    layer_bytes = work["w13"]["bytes"] + work["w2"]["bytes"] + work["route_permute"]["bytes"] + \
+        work["combine"]["bytes"]
+    layer_flops = work["w13"]["flops"] + work["w2"]["flops"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d_host = (wl.bf16_bits(x), logits.cpu().numpy(), wl.bf16_bits(w13), wl.bf16_bits(w2))
+        import oracle
+
+        v, sample, dt = oracle_sample(w, d_host, args.cpu_seconds)
+        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": f"{sample} in {dt:.1f} s"}
+
+    if rank == 0:
+        launches = moe.moe_forward_kernel_count(T, E, k, H, I)
+        line = {
+            "metric": metric_name(w),
+            "value": round(world * T / (ms / 1e3), 2),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": max(args.warmup, 3),
+            "ms_per_step": round(ms, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded; weights N(0,1/sqrt(fan_in)) random-init)",
+            "config": dict(w.as_dict(), parallelism=f"replicas{world}",
+                           tokens_per_rank=T, l2="flushed before every step (256 MiB write), "
+                           "outside the step events", n_touched_experts=n_touched),
+            "roofline": roof,
+            "layer": {"us": round(ms * 1e3, 2), "touched_bytes": layer_bytes,
+                      "GB/s": round(layer_bytes / (ms / 1e3) / 1e9, 1),
+                      "hbm_frac": round(layer_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                      "flops": layer_flops,
+                      "TFLOP/s": round(layer_flops / (ms / 1e3) / 1e12, 2),
+                      "stage_ms": {n: round(v, 5) for n, v in stage_ms.items()}},
+            "e2e": {"value": round(world * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 5)},
+            "cpu_baseline": cpu,
+            "gpu_launches": launches * (K + KB + KC + max(args.warmup, 3)),
+            "gpu_launches_timed_region": launches * K,
+            "clocks": clocks.report(),
+            "wall_s_timed_region": round(t_wall, 4),
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,153 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts layer forward.
+ *
+ * The layer (token t, expert e, top_k = k, hidden H, intermediate I):
+ *   route    : topk_ids[t, 0..k) = the k experts with the largest raw fp32 router
+ *              logit, ties to the lower expert index (-0.0 == +0.0), listed in
+ *              that order; topk_weights[t, j] = exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ *              over the selected logits ("softmax_sum" routing: FlashInfer PR #3751
+ *              page "Optimizing TRTLLM-Gen MoE routing", section "performance
+ *              numbers"; a softmax over all E followed by division by the sum of
+ *              the selected k is the same thing).
+ *   permute  : expanded row r = t*k + j.  expert_offsets[e+1] = expert_offsets[e] +
+ *              #{r : topk_ids[r] == e}; permuted_rows[expert_offsets[e] + q] = the
+ *              q-th smallest r routed to e (a stable sort by expert).
+ *   ffn      : for permuted position p of expert e, token t = permuted_rows[p] / k
+ *              (the `members[m] // input_route_divisor` map of the FlashInfer
+ *              PR #7368 page "overlap grouped activation staging", section
+ *              "1. Ampere", with the divisor equal to top_k):
+ *                h = w13[e] . x[t] (2I values), gate = h[0:I], up = h[I:2I],
+ *                act = silu(gate) * up  (silu(z) = z / (1 + exp(-z))),
+ *                y[permuted_rows[p]] = w2[e] . act  (H values).
+ *              The gate/up split of w13's rows is this library's reading: the
+ *              page elides its `split_gate` logic (section "2. Hopper").
+ *   combine  : out[t] = sum_{j=0..k-1} topk_weights[t, j] * y[t*k + j], in fp32,
+ *              j ascending, rounded once to bf16 (a fixed-order merge; cf. the
+ *              "FP32 partials" section of the FlashInfer PR #5586 page).
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is a DEVICE pointer to caller-owned memory, row-major
+ *     and contiguous.  The library never allocates, frees, synchronises (except
+ *     moe_device_status) or keeps a pointer past the completion of the call's
+ *     work on `stream`.
+ *   - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream).  Kernels are chained with programmatic
+ *     dependent launch; set MOE_DISABLE_PDL=1 in the environment to turn it off.
+ *   - All arguments are validated on the host before anything is launched; on an
+ *     error no work is queued and no output is touched:
+ *       NULL pointer                                      -> MOE_ERR_INVALID_ARG
+ *       T < 1, E < 1 or E > 1024, k < 1 or k > min(E, 16) -> MOE_ERR_UNSUPPORTED_SHAPE
+ *       (ffn/combine/forward) H or I < 128 or not a multiple of 128
+ *                                                         -> MOE_ERR_UNSUPPORTED_SHAPE
+ *       T*k > 2^30 or a size overflow                      -> MOE_ERR_UNSUPPORTED_SHAPE
+ *       a base pointer not 16-byte aligned                 -> MOE_ERR_MISALIGNED
+ *       ws_bytes < moe_workspace_size(shape)               -> MOE_ERR_WORKSPACE_TOO_SMALL
+ *     A failed launch returns MOE_ERR_CUDA; moe_last_cuda_error() then gives the
+ *     cudaError_t (per host thread).
+ *   - Inputs and outputs must not alias.  NaN logits are outside the contract.
+ *   - Element types: "bf16" is IEEE bfloat16 passed as its 16-bit pattern.
+ *   - The workspace is device memory of at least moe_workspace_size(shape) bytes,
+ *     256-byte aligned, owned by the caller; calls that share one workspace must
+ *     be ordered on one stream.  Its contents need no initialisation.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,
+    MOE_ERR_MISALIGNED = 3,
+    MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+    MOE_ERR_CUDA = 5,
+    MOE_ERR_DEVICE_TIMEOUT = 6
+} moe_status_t;
+
+/* T tokens, E experts, top_k, H hidden, I intermediate (H, I unused by route/permute). */
+typedef struct {
+    int32_t T, E, top_k, H, I;
+} moe_shape_t;
+
+typedef uint16_t moe_bf16_t;  /* bf16 bit pattern */
+typedef void* moe_stream_t;   /* cudaStream_t */
+
+/* Bytes of device workspace that moe_forward / moe_permute / moe_grouped_ffn need
+ * for `shape` (one size covers all three); 0 if the shape is unsupported.  Pure
+ * host function: touches no device. */
+size_t moe_workspace_size(moe_shape_t shape);
+
+/* route.  logits fp32 [T, E] -> topk_ids int32 [T, k], topk_weights fp32 [T, k]
+ * (both ordered by selection rank).  Needs no workspace. */
+moe_status_t moe_route(const float* logits, moe_shape_t shape, int32_t* topk_ids,
+                       float* topk_weights, moe_stream_t stream);
+
+/* permute.  topk_ids int32 [T*k] (values in [0, E)) -> expert_offsets int32 [E+1],
+ * permuted_rows int32 [T*k].  Ids outside [0, E) are outside the contract. */
+moe_status_t moe_permute(const int32_t* topk_ids, moe_shape_t shape, int32_t* expert_offsets,
+                         int32_t* permuted_rows, void* workspace, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* ffn.  x bf16 [T, H]; w13 bf16 [E, 2I, H]; w2 bf16 [E, H, I]; expert_offsets and
+ * permuted_rows as produced by moe_permute -> y bf16 [T*k, H] in expanded-id
+ * order (row r = t*k + j).  Activation rows are gathered straight from x (no
+ * permuted copy of x is made); gate/up accumulate in fp32 in tensor memory, act
+ * is rounded to bf16, the down projection accumulates in fp32 and y is rounded
+ * to bf16. */
+moe_status_t moe_grouped_ffn(const moe_bf16_t* x, const moe_bf16_t* w13, const moe_bf16_t* w2,
+                             const int32_t* expert_offsets, const int32_t* permuted_rows,
+                             moe_shape_t shape, moe_bf16_t* y, void* workspace, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* combine.  y bf16 [T*k, H] (expanded-id order), topk_weights fp32 [T, k]
+ * -> out bf16 [T, H].  Needs no workspace; shape.E and shape.I are not used. */
+moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_shape_t shape,
+                         moe_bf16_t* out, moe_stream_t stream);
+
+/* The whole layer: route -> permute -> ffn -> combine, one stream, no host sync.
+ * x bf16 [T, H], logits fp32 [T, E], w13 bf16 [E, 2I, H], w2 bf16 [E, H, I]
+ * -> out bf16 [T, H].  topk_ids, topk_weights, expert_offsets and permuted_rows
+ * are optional outputs: pass NULL to keep them inside the workspace. */
+moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
+                         const moe_bf16_t* w2, moe_shape_t shape, moe_bf16_t* out,
+                         int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
+                         int32_t* permuted_rows, void* workspace, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* moe_forward for measurement: identical work, and additionally records
+ * events[i] (cudaEvent_t, created by the caller) on `stream` at the stage
+ * boundaries: [0] before routing, [1] after route+permute, [2] after the
+ * w13/SwiGLU kernel, [3] after the w2 kernel, [4] after the combine.  n_events
+ * must be 5.  A recorded event is a stream operation, so the launch overlap
+ * between the stages it separates is lost while measuring. */
+moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
+                               const moe_bf16_t* w2, moe_shape_t shape, moe_bf16_t* out,
+                               int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
+                               int32_t* permuted_rows, void* workspace, size_t ws_bytes,
+                               moe_stream_t stream, void* const* events, int n_events);
+
+/* Number of kernels one moe_forward call launches for `shape` (0 if unsupported). */
+int moe_forward_kernel_count(moe_shape_t shape);
+
+/* Waits for `stream`, then reads and clears the device error word kept in the
+ * workspace.  MOE_ERR_DEVICE_TIMEOUT means a kernel gave up on a bounded
+ * intra-kernel wait (its outputs for that call are then unspecified). */
+moe_status_t moe_device_status(void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* The cudaError_t behind the last MOE_ERR_CUDA returned on this host thread. */
+int moe_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

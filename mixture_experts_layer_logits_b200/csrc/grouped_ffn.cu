@@ -1,0 +1,606 @@
+// grouped_ffn.cu -- the gathered grouped expert FFN on tcgen05 tensor cores.
+//
+// Two launches of one persistent, warp-specialised kernel template:
+//   w13 (MODE 0): act[p, f] = silu(gate) * up with gate/up = w13[e] rows f and
+//                 I + f dotted with x[permuted_rows[p] / k]; act is bf16 [R, I]
+//                 in permuted order.
+//   w2  (MODE 1): y[permuted_rows[p], h] = w2[e] row h dotted with act[p];
+//                 y is bf16 [R, H] in expanded-id order.
+//
+// Orientation ("swap AB", as on the FlashInfer PR #7368 page, section
+// "2. Hopper": weights are the TMA-fed operand, the few routed activation rows
+// the other one): the MMA's M = 128 rows are weight rows (output features), its
+// N = the routed token rows of one expert (16..256, rounded up to 16 per tile, so
+// a ragged tail costs at most 15 padded columns).  Accumulators live in tensor
+// memory (fp32); MODE 0 keeps a gate and an up accumulator of equal shape so the
+// epilogue thread that owns feature f holds both halves of its SwiGLU pair.
+//
+// Warp roles (256 threads):
+//   warp 0      TMA producer: weight tiles [128 x 64] (and, MODE 1, the act tile
+//               [NT x 64]) with the 128-byte swizzle into a STAGES-deep ring.
+//   warp 1      TMEM allocator and the single MMA-issuing thread.
+//   warps 2-3   MODE 0 activation gather: 16-byte cp.async of x rows selected by
+//               permuted_rows[p] / k straight into the swizzled B tile (no
+//               permuted copy of x exists), then fence.proxy.async and an
+//               mbarrier arrival -- the writer-side proxy fence and barrier the
+//               FlashInfer PR #7368 page ("2. Hopper") requires before an async
+//               proxy reads generic-proxy stores.  The weight TMA for a stage is
+//               issued independently of the gather, so the two overlap (the
+//               BF16 ordering of the same section).
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4) ..), SwiGLU / bf16 rounding / scatter, or split-K partials.
+//
+// Split-K: when there are too few (tile, feature block) units to fill the GPU
+// (decode), each unit's K range is cut into S slices; every slice writes an fp32
+// partial, and the CTA that finishes a unit last (an atomic arrival count, no
+// waiting) adds the S partials in slice order and runs the epilogue, so results
+// are bit-reproducible.
+//
+// Every mbarrier wait is bounded (mbar_wait); on a timeout the kernel records
+// an error word, stops issuing work, drains what it issued and frees TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;        // weight rows per tile (MMA M)
+constexpr int kBK = 64;         // K elements per stage (one 128-byte swizzle row)
+constexpr int kUmmaK = 16;      // K per tcgen05.mma (bf16)
+constexpr int kThreads = 256;
+constexpr int kATileBytes = kBM * kBK * 2;
+
+struct FfnArgs {
+    const __nv_bfloat16* x;
+    const int32_t* permuted_rows;
+    const Tile* tiles;
+    const int32_t* num_tiles;
+    __nv_bfloat16* out;       // MODE 0: act [R, I]; MODE 1: y [R, H]
+    float* partials;          // [S_max, R, pcols]
+    int32_t* counters;        // [fb_count, max_tiles]
+    int32_t* err;
+    int k, H, I, R;
+    int num_kt;               // K / 64
+    int fb_count;             // feature blocks of 128
+    int s_max;                // split-K upper bound
+    int max_tiles;
+    int min_kt_per_split;
+    int weights_evict_first;  // weights are streamed once (few tokens per expert)
+};
+
+template <int MODE, int NT>
+struct Cfg {
+    static constexpr int kNA = (MODE == 0) ? 2 : 1;               // A tiles per stage
+    static constexpr int kBTileBytes = NT * kBK * 2;
+    static constexpr int kStageBytes = kNA * kATileBytes + kBTileBytes;
+    static constexpr int kBudget = 220 * 1024;
+    static constexpr int kStagesRaw = kBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kAccCols = (MODE == 0) ? 2 * NT : NT;    // per accumulator buffer
+    static constexpr int kNBuf = (2 * kAccCols <= 512) ? 2 : 1;
+    static constexpr int kUsedCols = kAccCols * kNBuf;
+    static constexpr int kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64
+                                   : kUsedCols <= 128 ? 128 : kUsedCols <= 256 ? 256 : 512;
+    static constexpr uint32_t kTxBytes = kNA * kATileBytes + (MODE == 1 ? kBTileBytes : 0);
+    static constexpr int kGatherLag = (kStages - 1) < 3 ? (kStages - 1) : 3;
+    // shared memory: 1 KB alignment slack + ring + barriers/aux
+    static constexpr int kAuxBytes = 1024 + 2 * NT * 4;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kAuxBytes;
+    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N tile");
+    static_assert(kStages >= 2, "pipeline depth");
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+};
+
+struct Aux {
+    uint64_t full[16];
+    uint64_t empty[16];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int last;
+    int pad;
+};
+
+__device__ __forceinline__ int split_count(const FfnArgs& a, int ntiles)
+{
+    // enough (tile, feature block, slice) units for ~16 waves of CTAs, each slice
+    // at least min_kt_per_split K tiles long
+    const int units = ntiles * a.fb_count;
+    if (units <= 0) return 1;
+    int s = (16 * (int)gridDim.x + units - 1) / units;
+    s = min(s, a.s_max);
+    s = min(s, max(1, a.num_kt / a.min_kt_per_split));
+    return max(s, 1);
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+__device__ __forceinline__ void named_bar_sync(int id, int n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// bar.red.or over `n` threads: true in every thread if any thread passed true.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
+
+__device__ __forceinline__ void flag_error(const FfnArgs& a, Aux* aux)
+{
+    atomicExch(a.err, kDeviceErrorMagic);
+    aux->abort = 1;
+}
+
+template <int MODE, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_act, const FfnArgs a)
+{
+    using C = Cfg<MODE, NT>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    Aux* aux = reinterpret_cast<Aux*>(ring + C::kStages * C::kStageBytes);
+    int* tok_off = reinterpret_cast<int*>(aux + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&aux->full[s], MODE == 0 ? 1 + 64 : 1);
+            mbar_init(&aux->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&aux->tfull[b], 1);
+            mbar_init(&aux->tempty[b], 4);
+        }
+        mbar_init(&aux->drain, 1);
+        aux->abort = 0;
+        aux->last = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_w);
+        if (MODE == 1) tma_prefetch_desc(&tm_act);
+    }
+    if (warp == 1) {
+        tmem_alloc(&aux->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = aux->tmem_base;
+
+    pdl_wait();  // routing, permutation, tile list (and, MODE 1, act) are ready
+    pdl_launch_dependents();
+
+    const int ntiles = *a.num_tiles;
+    const int s_want = split_count(a, ntiles);
+    const int kt_per_split = (a.num_kt + s_want - 1) / s_want;
+    const int S = (a.num_kt + kt_per_split - 1) / kt_per_split;  // every slice non-empty
+    const int units = ntiles * a.fb_count * S;
+    volatile int* abort_flag = &aux->abort;
+
+    // unit u -> (slice, tile, feature block); adjacent units share a weight block
+    auto decode = [&](int u, int& split, int& tile, int& fb) {
+        split = u % S;
+        const int rest = u / S;
+        tile = rest % ntiles;
+        fb = rest / ntiles;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol = a.weights_evict_first ? l2_policy_evict_first()
+                                                       : l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[16];
+            for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int split, tile, fb;
+                decode(u, split, tile, fb);
+                const Tile t = a.tiles[tile];
+                const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (!mbar_wait(&aux->empty[stage], phase ^ 1u, abort_flag)) {
+                        flag_error(a, aux);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = ring + stage * C::kStageBytes;
+                    mbar_arrive_expect_tx(&aux->full[stage], C::kTxBytes);
+                    if (MODE == 0) {
+                        const int row = t.expert * 2 * a.I + fb * kBM;
+                        tma_load_2d(st, &tm_w, &aux->full[stage], kt * kBK, row, pol);
+                        tma_load_2d(st + kATileBytes, &tm_w, &aux->full[stage], kt * kBK, row + a.I,
+                                    pol);
+                    } else {
+                        const int row = t.expert * a.H + fb * kBM;
+                        tma_load_2d(st, &tm_w, &aux->full[stage], kt * kBK, row, pol);
+                        tma_load_2d_nohint(st + kATileBytes, &tm_act, &aux->full[stage], kt * kBK,
+                                           t.row_start);
+                    }
+                    issued[stage] += 1;
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok || *abort_flag) {
+                // let every TMA load already issued land before the CTA can exit
+                for (int s = 0; s < C::kStages; ++s)
+                    if (issued[s] > 0) {
+                        volatile int never = 0;
+                        mbar_wait(&aux->full[s], (uint32_t)((issued[s] - 1) & 1), &never,
+                                  500000000ull);
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int lu = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++lu) {
+                int split, tile, fb;
+                decode(u, split, tile, fb);
+                const Tile t = a.tiles[tile];
+                const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
+                const int b = (C::kNBuf == 2) ? (lu & 1) : 0;
+                const uint32_t aphase = (uint32_t)((C::kNBuf == 2 ? (lu >> 1) : lu) & 1);
+                if (!mbar_wait(&aux->tempty[b], aphase ^ 1u, abort_flag)) {
+                    flag_error(a, aux);
+                    break;
+                }
+                tc_fence_after();
+                const int n = (t.rows + 15) & ~15;
+                const uint32_t idesc = umma_idesc_bf16(kBM, n);
+                const uint32_t d0 = tmem_base + (uint32_t)(b * C::kAccCols);
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (!mbar_wait(&aux->full[stage], phase, abort_flag)) {
+                        flag_error(a, aux);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(ring + stage * C::kStageBytes);
+                    const uint32_t bt = st + C::kNA * kATileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        const uint32_t acc = (kt > kt0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
+                        umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
+                        if (MODE == 0)
+                            umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
+                                      idesc, acc);
+                    }
+                    umma_commit(&aux->empty[stage]);  // frees the smem stage when read
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) umma_commit(&aux->tfull[b]);
+            }
+            // all MMAs issued by this thread are complete before TMEM is freed
+            umma_commit(&aux->drain);
+            volatile int never = 0;
+            if (!mbar_wait(&aux->drain, 0, &never, 500000000ull)) atomicExch(a.err, kDeviceErrorMagic);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ gather (MODE 0)
+        if (MODE == 0) {
+            const int gt = threadIdx.x - 64;  // 0..63
+            constexpr int kLag = C::kGatherLag;
+            int ring_stage[4];
+            int issued = 0, arrived = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int split, tile, fb;
+                decode(u, split, tile, fb);
+                const Tile t = a.tiles[tile];
+                const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
+                // each gather warp keeps its own copy of the tile's token offsets
+                int* my_off = tok_off + (warp - 2) * NT;
+                __syncwarp();  // previous unit's offsets are no longer read
+                for (int j = lane; j < t.rows; j += 32)
+                    my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
+                __syncwarp();
+                const int chunks = t.rows * 8;
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    // warp-uniform decision, so no lane is left behind at __syncwarp
+                    if (!__all_sync(0xffffffffu, mbar_wait(&aux->empty[stage], phase ^ 1u,
+                                                           abort_flag))) {
+                        if (lane == 0) flag_error(a, aux);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bt =
+                        smem_u32(ring + stage * C::kStageBytes + C::kNA * kATileBytes);
+                    const __nv_bfloat16* src0 = a.x + kt * kBK;
+                    for (int q = gt; q < chunks; q += 64) {
+                        const int j = q >> 3, c = q & 7;
+                        cp_async_16(bt + j * 128 + ((c ^ (j & 7)) << 4), src0 + my_off[j] + c * 8);
+                    }
+                    cp_async_commit();
+                    ring_stage[issued & 3] = stage;
+                    ++issued;
+                    if (issued - arrived > kLag) {
+                        cp_async_wait<kLag>();
+                        fence_proxy_async_smem();
+                        while (issued - arrived > kLag) mbar_arrive(&aux->full[ring_stage[arrived++ & 3]]);
+                    }
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            while (arrived < issued) mbar_arrive(&aux->full[ring_stage[arrived++ & 3]]);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int f_local = q * 32 + lane;      // feature inside the 128-row block
+        const int pcols = (MODE == 0) ? 2 * a.I : a.H;
+        const int ocols = (MODE == 0) ? a.I : a.H;
+        int lu = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++lu) {
+            int split, tile, fb;
+            decode(u, split, tile, fb);
+            const Tile t = a.tiles[tile];
+            const int b = (C::kNBuf == 2) ? (lu & 1) : 0;
+            const uint32_t aphase = (uint32_t)((C::kNBuf == 2 ? (lu >> 1) : lu) & 1);
+            const bool got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
+            if (!got) flag_error(a, aux);
+            if (named_bar_or(1, 128, !got || *abort_flag)) break;  // same decision in all 4 warps
+            tc_fence_after();
+            const int f = fb * kBM + f_local;
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols);
+            for (int j0 = 0; j0 < t.rows; j0 += 16) {
+                uint32_t g[16], v[16];
+                tmem_ld16(tacc + j0, g);
+                if (MODE == 0) tmem_ld16(tacc + NT + j0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = j0 + jj;
+                    if (j >= t.rows) break;
+                    const int p = t.row_start + j;
+                    const float gv = __uint_as_float(g[jj]);
+                    if (S == 1) {
+                        if (MODE == 0) {
+                            a.out[(size_t)p * ocols + f] =
+                                __float2bfloat16_rn(silu_mul(gv, __uint_as_float(v[jj])));
+                        } else {
+                            const int r = a.permuted_rows[p];
+                            a.out[(size_t)r * ocols + f] = __float2bfloat16_rn(gv);
+                        }
+                    } else {
+                        float* prow = a.partials + ((size_t)split * a.R + p) * pcols;
+                        prow[f] = gv;
+                        if (MODE == 0) prow[a.I + f] = __uint_as_float(v[jj]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&aux->tempty[b]);
+
+            if (S > 1) {
+                // the CTA that completes a unit's last slice reduces all slices in order
+                __threadfence();
+                named_bar_sync(1, 128);
+                const int cidx = fb * a.max_tiles + tile;
+                if (threadIdx.x == 128) aux->last = (atomicAdd(&a.counters[cidx], 1) == S - 1);
+                named_bar_sync(1, 128);
+                if (aux->last) {
+                    __threadfence();
+                    for (int j = 0; j < t.rows; ++j) {
+                        const int p = t.row_start + j;
+                        float gs = 0.f, us = 0.f;
+                        for (int s = 0; s < S; ++s) {
+                            const float* prow = a.partials + ((size_t)s * a.R + p) * pcols;
+                            gs += ld_cg(prow + f);
+                            if (MODE == 0) us += ld_cg(prow + a.I + f);
+                        }
+                        if (MODE == 0) {
+                            a.out[(size_t)p * ocols + f] = __float2bfloat16_rn(silu_mul(gs, us));
+                        } else {
+                            const int r = a.permuted_rows[p];
+                            a.out[(size_t)r * ocols + f] = __float2bfloat16_rn(gs);
+                        }
+                    }
+                    if (threadIdx.x == 128) a.counters[cidx] = 0;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2D bf16 row-major [rows, cols] tensor map with a [box_rows, 64] box, 128-byte swizzle.
+cudaError_t make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE, int NT>
+cudaError_t launch_mode(const CUtensorMap& tw, const CUtensorMap& ta, const FfnArgs& a, int grid,
+                        cudaStream_t st)
+{
+    using C = Cfg<MODE, NT>;
+    auto kern = grouped_gemm_kernel<MODE, NT>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tw, ta, a);
+}
+
+template <int MODE>
+cudaError_t launch_nt(int nt, const CUtensorMap& tw, const CUtensorMap& ta, const FfnArgs& a,
+                      int grid, cudaStream_t st)
+{
+    switch (nt) {
+    case 16: return launch_mode<MODE, 16>(tw, ta, a, grid, st);
+    case 32: return launch_mode<MODE, 32>(tw, ta, a, grid, st);
+    case 64: return launch_mode<MODE, 64>(tw, ta, a, grid, st);
+    case 128: return launch_mode<MODE, 128>(tw, ta, a, grid, st);
+    case 256: return launch_mode<MODE, 256>(tw, ta, a, grid, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+FfnPlan plan_ffn(int T, int E, int k, int H, int I, int num_sms)
+{
+    FfnPlan p;
+    const long R = (long)T * k;
+    // one tile per expert whenever an expert can hold every token (each token
+    // picks an expert at most once), so decode streams each weight block once
+    int nt = 16;
+    while (nt < 256 && nt < T) nt *= 2;
+    p.nt = nt;
+    p.max_tiles = (int)((R + nt - 1) / nt + (E < R ? E : R));
+    // split-K only pays when even the smallest possible tile count leaves the GPU idle
+    const long min_units13 = ((R + nt - 1) / nt) * (I / kBM);
+    const long min_units2 = ((R + nt - 1) / nt) * (H / kBM);
+    const long target = 16L * num_sms;
+    p.s13_max = min_units13 >= target ? 1 : 8;
+    p.s2_max = min_units2 >= target ? 1 : 8;
+    p.grid = num_sms;
+    return p;
+}
+
+cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, int I,
+                               const FfnPlan& plan, cudaStream_t st, cudaEvent_t between_gemms)
+{
+    const int R = T * k;
+    CUtensorMap tw13, tw2, tact;
+    cudaError_t err = make_tmap(&tw13, b.w13, (uint64_t)E * 2 * I, (uint64_t)H, kBM);
+    if (err == cudaSuccess) err = make_tmap(&tw2, b.w2, (uint64_t)E * H, (uint64_t)I, kBM);
+    if (err == cudaSuccess) err = make_tmap(&tact, b.act, (uint64_t)R, (uint64_t)I, (uint32_t)plan.nt);
+    if (err != cudaSuccess) return err;
+
+    FfnArgs a = {};
+    a.x = static_cast<const __nv_bfloat16*>(b.x);
+    a.permuted_rows = b.permuted_rows;
+    a.tiles = b.tiles;
+    a.num_tiles = b.num_tiles;
+    a.partials = b.partials;
+    a.err = b.err;
+    a.k = k;
+    a.H = H;
+    a.I = I;
+    a.R = R;
+    a.max_tiles = plan.max_tiles;
+    a.min_kt_per_split = 4;
+    a.weights_evict_first = plan.nt <= 64 ? 1 : 0;
+
+    // w13 + SwiGLU: K = H
+    a.out = static_cast<__nv_bfloat16*>(b.act);
+    a.counters = b.counters13;
+    a.num_kt = H / kBK;
+    a.fb_count = I / kBM;
+    a.s_max = plan.s13_max;
+    err = launch_nt<0>(plan.nt, tw13, tw13, a, plan.grid, st);
+    if (err != cudaSuccess) return err;
+    if (between_gemms) {
+        err = cudaEventRecord(between_gemms, st);
+        if (err != cudaSuccess) return err;
+    }
+
+    // w2: K = I
+    a.out = static_cast<__nv_bfloat16*>(b.y);
+    a.counters = b.counters2;
+    a.num_kt = I / kBK;
+    a.fb_count = H / kBM;
+    a.s_max = plan.s2_max;
+    return launch_nt<1>(plan.nt, tw2, tact, a, plan.grid, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,90 @@
+// kernels.h -- host-side launch interface between the C ABI (moe_api.cu) and the
+// kernels (route_permute.cu, grouped_ffn.cu, combine.cu).  Internal only.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Value a kernel stores in the workspace's error word when it gives up on a
+// bounded wait.  A fresh workspace holds arbitrary bytes, so only this exact
+// value counts as an error.
+constexpr int32_t kDeviceErrorMagic = 0x4D4F4554;
+
+// One tile of the grouped GEMMs: `rows` (1..NT) consecutive permuted rows of one
+// expert, starting at permuted position `row_start`.
+struct Tile {
+    int expert;
+    int row_start;
+    int rows;
+    int pad;
+};
+
+// Everything the route/permute kernels write besides the user-visible outputs.
+struct PermuteAux {
+    Tile* tiles;           // [max_tiles]
+    int32_t* num_tiles;    // device scalar
+    int nt;                // token rows per tile (the GEMM's N tile)
+    int32_t* counters;     // split-K arrival counters to zero, [n_counters]
+    int n_counters;
+    int32_t* chunk_counts; // [n_chunks, E] scratch of the multi-CTA path
+};
+
+// Launch helper: programmatic dependent launch unless MOE_DISABLE_PDL=1.
+bool pdl_enabled();
+
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights,
+                         cudaStream_t st);
+
+// Single-CTA path (T*k <= kSmallRows): optional routing, then histogram, scan,
+// stable scatter, tile list.  logits == nullptr: ids are an input.
+constexpr int kSmallRows = 4096;
+cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k, int32_t* ids,
+                                       float* weights, int32_t* offsets, int32_t* rows,
+                                       const PermuteAux& aux, cudaStream_t st);
+
+// Multi-CTA path: per-chunk counts, a scan over (expert, chunk), a per-chunk
+// stable scatter, tile list.
+constexpr int kChunkRows = 4096;
+cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
+                                 int32_t* rows, const PermuteAux& aux, cudaStream_t st);
+size_t large_permute_smem(int E);
+
+// Tile list from expert_offsets alone (moe_grouped_ffn called on its own).
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, const PermuteAux& aux,
+                               cudaStream_t st);
+
+struct FfnPlan {
+    int nt;            // token rows per tile (16..256, multiple of 16)
+    int max_tiles;     // upper bound of the tile count
+    int s13_max;       // split-K bounds (device picks the actual split)
+    int s2_max;
+    int grid;          // persistent CTAs
+};
+FfnPlan plan_ffn(int T, int E, int k, int H, int I, int num_sms);
+
+struct FfnBuffers {
+    const void* x;
+    const void* w13;
+    const void* w2;
+    const int32_t* permuted_rows;
+    const Tile* tiles;
+    const int32_t* num_tiles;
+    void* act;         // bf16 [R, I]
+    void* y;           // bf16 [R, H]
+    float* partials;   // fp32 split-K partials
+    int32_t* counters13;
+    int32_t* counters2;
+    int32_t* err;
+};
+// between_gemms: if not null, recorded on `st` after the w13 launch.
+cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, int I,
+                               const FfnPlan& plan, cudaStream_t st,
+                               cudaEvent_t between_gemms = nullptr);
+
+cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
+                           cudaStream_t st);
+
+}  // namespace moe

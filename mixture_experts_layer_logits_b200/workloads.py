@@ -113,17 +113,22 @@ def make_x(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
     return torch.randn(w.T, w.H, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
 
 
+def make_expert_weights(w: Workload, e: int, seed: int = 0, device="cpu"):
+    """(w13[e] bf16 [2I,H], w2[e] bf16 [H,I]) of one expert; each expert has its own
+    generator, so one expert can be drawn without the others."""
+    g13 = _gen(device, seed * 65_537 + e, _TAG_W13)
+    g2 = _gen(device, seed * 65_537 + e, _TAG_W2)
+    a = (torch.randn(2 * w.I, w.H, generator=g13, device=device) / math.sqrt(w.H))
+    b = (torch.randn(w.H, w.I, generator=g2, device=device) / math.sqrt(w.I))
+    return a.to(torch.bfloat16), b.to(torch.bfloat16)
+
+
 def make_weights(w: Workload, seed: int = 0, device="cpu"):
     """(w13 bf16 [E,2I,H], w2 bf16 [E,H,I]), drawn one expert at a time."""
     w13 = torch.empty(w.E, 2 * w.I, w.H, dtype=torch.bfloat16, device=device)
     w2 = torch.empty(w.E, w.H, w.I, dtype=torch.bfloat16, device=device)
-    g13 = _gen(device, seed, _TAG_W13)
-    g2 = _gen(device, seed, _TAG_W2)
-    s13 = 1.0 / math.sqrt(w.H)
-    s2 = 1.0 / math.sqrt(w.I)
     for e in range(w.E):
-        w13[e] = (torch.randn(2 * w.I, w.H, generator=g13, device=device) * s13).to(torch.bfloat16)
-        w2[e] = (torch.randn(w.H, w.I, generator=g2, device=device) * s2).to(torch.bfloat16)
+        w13[e], w2[e] = make_expert_weights(w, e, seed, device)
     return w13, w2
 
 

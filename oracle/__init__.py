@@ -46,7 +46,8 @@ def _load():
     lib.oracle_forward_tokens.argtypes = [_u16p, _f32p, ctypes.POINTER(_u16p),
                                           ctypes.POINTER(_u16p), i, i, i, i, i, i, i, _i32p,
                                           _f64p]
-    for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_ffn, lib.oracle_combine,
+    lib.oracle_num_threads.argtypes = []
+    for fn in (lib.oracle_num_threads, lib.oracle_route, lib.oracle_permute, lib.oracle_ffn, lib.oracle_combine,
                lib.oracle_forward, lib.oracle_forward_tokens):
         fn.restype = ctypes.c_int
     _lib = lib
@@ -67,6 +68,11 @@ def _c(a, dtype):
 def _check(rc, name):
     if rc != 0:
         raise ValueError(f"{name} rejected its arguments (rc={rc})")
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (OMP_NUM_THREADS, else the host's cores)."""
+    return int(_load().oracle_num_threads())
 
 
 def route(logits: np.ndarray, k: int):

@@ -41,9 +41,13 @@
  * SwiGLU MLP, and a dense all-experts masked loop).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+
+/* Number of OpenMP threads the oracle's parallel loops use. */
+int oracle_num_threads(void) { return omp_get_max_threads(); }
 
 /* ---- exact upcasts ------------------------------------------------------ */
 
