@@ -132,6 +132,31 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
                                int32_t* permuted_rows, void* workspace, size_t ws_bytes,
                                moe_stream_t stream, void* const* events, int n_events);
 
+/* moe_permute without a workspace argument, for callers that cannot allocate
+ * device memory: code that must not grow its device footprint after start-up,
+ * code whose device memory is all owned by another allocator, or callers that
+ * are handed only the input and output buffers.  The FlashInfer pages have no
+ * counterpart of this entry point; it computes exactly what moe_permute
+ * computes (same kernels, same bit-exact result).
+ *
+ * Scratch: a file-scope device array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES
+ * (about 1 MiB) inside the library; every GPU on which the library is used holds
+ * it until the process exits.  The caller still passes topk_ids, expert_offsets
+ * and permuted_rows (device pointers, 16-byte aligned).
+ * Limits: T*k <= MOE_PERMUTE_NOALLOC_MAX_ROWS and the moe_permute shape rules,
+ * else MOE_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ * The first call on each device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.
+ * Every call shares the one array: calls whose GPU work can overlap (on other
+ * streams or host threads, same device) race and may return wrong results;
+ * order them on one stream. */
+#define MOE_PERMUTE_NOALLOC_MAX_ROWS (1 << 20)
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (1048576 + 16384 + 256)
+moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
+                                 int32_t* expert_offsets, int32_t* permuted_rows,
+                                 moe_stream_t stream);
+
 /* Number of kernels one moe_forward call launches for `shape` (0 if unsupported). */
 int moe_forward_kernel_count(moe_shape_t shape);
 

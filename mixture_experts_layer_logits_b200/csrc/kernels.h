@@ -32,6 +32,9 @@ struct PermuteAux {
     int32_t* chunk_counts; // [n_chunks, E] scratch of the multi-CTA path
 };
 
+// Records the cudaError_t that moe_last_cuda_error() reports on this host thread.
+void set_last_cuda_error(int err);
+
 // Launch helper: programmatic dependent launch unless MOE_DISABLE_PDL=1.
 bool pdl_enabled();
 

@@ -23,8 +23,12 @@ bool pdl_enabled()
 }
 
 namespace {
-
 thread_local int g_last_cuda_error = 0;
+}  // namespace
+
+void set_last_cuda_error(int err) { g_last_cuda_error = err; }
+
+namespace {
 
 // Plans and workspaces are sized for the B200's SM count; the launch grid uses
 // the actual device's.
