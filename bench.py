@@ -55,12 +55,24 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="decode")
+    p.add_argument("--workload", default="decode",
+                   help="a named workload, or custom:T=..,E=..,k=..,H=..,I=..[,zipf=..]")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the cpu_baseline sample")
     return p.parse_args(argv)
+
+
+def get_workload(spec):
+    from mixture_experts_layer_logits_b200 import workloads as wl
+
+    if not spec.startswith("custom:"):
+        return wl.WORKLOADS[spec]
+    kv = dict(item.split("=") for item in spec[len("custom:"):].split(","))
+    return wl.custom(spec, int(kv["T"]), int(kv["E"]), int(kv["k"]), int(kv.get("H", 0)),
+                     int(kv.get("I", 0)), zipf_s=float(kv.get("zipf", 0.0)),
+                     dup_frac=float(kv.get("dup", 0.0)))
 
 
 def dist_env():
@@ -220,7 +232,7 @@ def reference_arm(args, rank, world):
     import oracle
     from mixture_experts_layer_logits_b200 import workloads as wl
 
-    w = wl.WORKLOADS[args.workload]
+    w = get_workload(args.workload)
     d = wl.make_inputs(w, seed=args.seed, device="cpu", weights=False)
     logits = d["logits"].numpy()
     cfg = dict(w.as_dict())
@@ -273,6 +285,132 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def routing_bench(args, w, rank, world, local, dev, pg):
+    """Routing-only workload: a step is moe_route + moe_permute over T tokens."""
+    import torch
+
+    import mixture_experts_layer_logits_b200 as moe
+    from mixture_experts_layer_logits_b200 import workloads as wl
+
+    T, E, k = w.T, w.E, w.k
+    R = T * k
+    logits = wl.make_logits(w, seed=args.seed + rank, device=dev)
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    wts = torch.empty(T, k, dtype=torch.float32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    rows = torch.empty(R, dtype=torch.int32, device=dev)
+    ws = moe.workspace(T, E, k, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        moe.moe_route(logits, k, topk_ids=ids, topk_weights=wts)
+        if evs:
+            evs[1].record(stream)
+        moe.moe_permute(ids, E, ws=ws, expert_offsets=off, permuted_rows=rows)
+        if evs:
+            evs[2].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+
+    def max_over_ranks(v):
+        if not pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    W = max(args.warmup, 3)
+    for _ in range(W):
+        flush.zero_()
+        step()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier()
+    with ClockSampler(local) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(K):
+            flush.zero_()
+            step(ev[i])
+        barrier()
+        t_wall = time.perf_counter() - t_wall
+    ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
+    route_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    perm_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+
+    # e2e: logits from pinned host memory in, the four outputs back out
+    logits_h = logits.cpu().pin_memory()
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (ids, wts, off, rows)]
+    KC = min(K, 200)
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(KC)]
+    barrier()
+    for i in range(KC):
+        flush.zero_()
+        eev[i][0].record(stream)
+        logits.copy_(logits_h, non_blocking=True)
+        step()
+        for h, d in zip(outs_h, (ids, wts, off, rows)):
+            h.copy_(d, non_blocking=True)
+        eev[i][1].record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in eev))
+
+    peaks, peak_kind = load_peaks()
+    route_bytes = T * E * 4 + R * 8
+    perm_bytes = R * 4 + (E + 1) * 4 + R * 4
+    dominant, dom_ms, dom_bytes = ("route", route_ms, route_bytes) if route_ms >= perm_ms else \
+        ("permute", perm_ms, perm_bytes)
+    roof = roofline_entry(dominant, dict(bytes=dom_bytes, flops=0), dom_ms, peaks, peak_kind,
+                          False, NCU_TRAFFIC.get((w.name, dominant)))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        lg = logits.cpu().numpy()
+        n = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            rid, _ = oracle.route(lg, k)
+            oracle.permute(rid, E)
+            n += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": round(n * T / dt, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": f"all {T} tokens (route + permute) x {n} in {dt:.1f} s"}
+    if rank == 0:
+        all_bytes = route_bytes + perm_bytes
+        launches = 1 + (1 if R <= 4096 else 3)
+        line = {
+            "metric": metric_name(w), "value": round(world * T / (ms / 1e3), 2),
+            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
+            "config": dict(w.as_dict(), parallelism=f"replicas{world}",
+                           l2="flushed before every step (256 MiB write), outside the step events"),
+            "roofline": roof,
+            "stage_ms": {"route": round(route_ms, 5), "permute": round(perm_ms, 5)},
+            "step_GB/s": round(all_bytes / (ms / 1e3) / 1e9, 1),
+            "e2e": {"value": round(world * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": logits_h.numel() * 4,
+                    "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in outs_h),
+                    "ms_per_step": round(e2e_ms, 5)},
+            "cpu_baseline": cpu,
+            "gpu_launches": launches * (K + KC + W),
+            "gpu_launches_timed_region": launches * K,
+            "clocks": clocks.report(),
+            "wall_s_timed_region": round(t_wall, 4),
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
 def metric_name(w):
     return ("MoE layer forward tokens/s at 1 B200 (us/layer in ms_per_step)" if w.has_ffn
             else "MoE routing (route + permute) tokens/s at 1 B200")
@@ -309,9 +447,9 @@ def main(argv=None):
         dist.barrier()
     moe.load_library()
 
-    w = wl.WORKLOADS[args.workload]
+    w = get_workload(args.workload)
     if not w.has_ffn:
-        raise SystemExit("bench.py times the whole layer; pick a workload with an FFN")
+        return routing_bench(args, w, rank, world, local, dev, pg)
     T, E, k, H, I = w.T, w.E, w.k, w.H, w.I
     R = T * k
     # this rank's tokens; weights are the same on every rank

@@ -31,10 +31,11 @@
 //               32*(w%4) ..), SwiGLU / bf16 rounding / scatter, or split-K partials.
 //
 // Split-K: when there are too few (tile, feature block) units to fill the GPU
-// (decode), each unit's K range is cut into S slices; every slice writes an fp32
-// partial, and the CTA that finishes a unit last (an atomic arrival count, no
-// waiting) adds the S partials in slice order and runs the epilogue, so results
-// are bit-reproducible.
+// (decode), each unit's K range is cut into S slices (S chosen on the device
+// from the tile count and written to the workspace).  Every slice stores its
+// fp32 partial with plain stores and moves on -- no fence, atomic or wait on the
+// critical path.  The slices are added in slice order later, by the SwiGLU
+// finalize kernel (w13) and by the combine (w2), so results are bit-reproducible.
 //
 // Every mbarrier wait is bounded (mbar_wait); on a timeout the kernel records
 // an error word, stops issuing work, drains what it issued and frees TMEM.
@@ -65,8 +66,8 @@ struct FfnArgs {
     const Tile* tiles;
     const int32_t* num_tiles;
     __nv_bfloat16* out;       // MODE 0: act [R, I]; MODE 1: y [R, H]
-    float* partials;          // [S_max, R, pcols]
-    int32_t* counters;        // [fb_count, max_tiles]
+    float* partials;          // MODE 0: [S, R, 2I] by permuted row; MODE 1: [S, R, H] by expanded id
+    int32_t* split_out;       // CTA 0 records the split count S here
     int32_t* err;
     int k, H, I, R;
     int num_kt;               // K / 64
@@ -86,7 +87,8 @@ struct Cfg {
     static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kAccCols = (MODE == 0) ? 2 * NT : NT;    // per accumulator buffer
-    static constexpr int kNBuf = (2 * kAccCols <= 512) ? 2 : 1;
+    static constexpr int kNBufRaw = 512 / kAccCols;                // accumulators in flight
+    static constexpr int kNBuf = kNBufRaw > 8 ? 8 : kNBufRaw;
     static constexpr int kUsedCols = kAccCols * kNBuf;
     static constexpr int kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64
                                    : kUsedCols <= 128 ? 128 : kUsedCols <= 256 ? 256 : 512;
@@ -103,8 +105,8 @@ struct Cfg {
 struct Aux {
     uint64_t full[16];
     uint64_t empty[16];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t tfull[8];
+    uint64_t tempty[8];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&aux->full[s], MODE == 0 ? 1 + 64 : 1);
             mbar_init(&aux->empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::kNBuf; ++b) {
             mbar_init(&aux->tfull[b], 1);
             mbar_init(&aux->tempty[b], 4);
         }
@@ -203,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kt_per_split = (a.num_kt + s_want - 1) / s_want;
     const int S = (a.num_kt + kt_per_split - 1) / kt_per_split;  // every slice non-empty
     const int units = ntiles * a.fb_count * S;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.split_out = S;
     volatile int* abort_flag = &aux->abort;
 
     // unit u -> (slice, tile, feature block); adjacent units share a weight block
@@ -276,8 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode(u, split, tile, fb);
                 const Tile t = a.tiles[tile];
                 const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
-                const int b = (C::kNBuf == 2) ? (lu & 1) : 0;
-                const uint32_t aphase = (uint32_t)((C::kNBuf == 2 ? (lu >> 1) : lu) & 1);
+                const int b = lu % C::kNBuf;
+                const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
                 if (!mbar_wait(&aux->tempty[b], aphase ^ 1u, abort_flag)) {
                     flag_error(a, aux);
                     break;
@@ -383,8 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int split, tile, fb;
             decode(u, split, tile, fb);
             const Tile t = a.tiles[tile];
-            const int b = (C::kNBuf == 2) ? (lu & 1) : 0;
-            const uint32_t aphase = (uint32_t)((C::kNBuf == 2 ? (lu >> 1) : lu) & 1);
+            const int b = lu % C::kNBuf;
+            const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
             const bool got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
             if (!got) flag_error(a, aux);
             if (named_bar_or(1, 128, !got || *abort_flag)) break;  // same decision in all 4 warps
@@ -410,44 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int r = a.permuted_rows[p];
                             a.out[(size_t)r * ocols + f] = __float2bfloat16_rn(gv);
                         }
-                    } else {
+                    } else if (MODE == 0) {
                         float* prow = a.partials + ((size_t)split * a.R + p) * pcols;
                         prow[f] = gv;
-                        if (MODE == 0) prow[a.I + f] = __uint_as_float(v[jj]);
+                        prow[a.I + f] = __uint_as_float(v[jj]);
+                    } else {
+                        const int r = a.permuted_rows[p];
+                        a.partials[((size_t)split * a.R + r) * pcols + f] = gv;
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&aux->tempty[b]);
-
-            if (S > 1) {
-                // the CTA that completes a unit's last slice reduces all slices in order
-                __threadfence();
-                named_bar_sync(1, 128);
-                const int cidx = fb * a.max_tiles + tile;
-                if (threadIdx.x == 128) aux->last = (atomicAdd(&a.counters[cidx], 1) == S - 1);
-                named_bar_sync(1, 128);
-                if (aux->last) {
-                    __threadfence();
-                    for (int j = 0; j < t.rows; ++j) {
-                        const int p = t.row_start + j;
-                        float gs = 0.f, us = 0.f;
-                        for (int s = 0; s < S; ++s) {
-                            const float* prow = a.partials + ((size_t)s * a.R + p) * pcols;
-                            gs += ld_cg(prow + f);
-                            if (MODE == 0) us += ld_cg(prow + a.I + f);
-                        }
-                        if (MODE == 0) {
-                            a.out[(size_t)p * ocols + f] = __float2bfloat16_rn(silu_mul(gs, us));
-                        } else {
-                            const int r = a.permuted_rows[p];
-                            a.out[(size_t)r * ocols + f] = __float2bfloat16_rn(gs);
-                        }
-                    }
-                    if (threadIdx.x == 128) a.counters[cidx] = 0;
-                }
-            }
         }
     }
 
@@ -583,12 +561,16 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
 
     // w13 + SwiGLU: K = H
     a.out = static_cast<__nv_bfloat16*>(b.act);
-    a.counters = b.counters13;
+    a.split_out = b.splits;
     a.num_kt = H / kBK;
     a.fb_count = I / kBM;
     a.s_max = plan.s13_max;
     err = launch_nt<0>(plan.nt, tw13, tw13, a, plan.grid, st);
     if (err != cudaSuccess) return err;
+    if (plan.s13_max > 1) {
+        err = launch_swiglu_finalize(b.partials, b.splits, R, I, b.act, st);
+        if (err != cudaSuccess) return err;
+    }
     if (between_gemms) {
         err = cudaEventRecord(between_gemms, st);
         if (err != cudaSuccess) return err;
@@ -596,7 +578,7 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
 
     // w2: K = I
     a.out = static_cast<__nv_bfloat16*>(b.y);
-    a.counters = b.counters2;
+    a.split_out = b.splits + 1;
     a.num_kt = I / kBK;
     a.fb_count = H / kBM;
     a.s_max = plan.s2_max;

@@ -62,7 +62,7 @@ cudaError_t launch_build_tiles(const int32_t* offsets, int E, const PermuteAux& 
 struct FfnPlan {
     int nt;            // token rows per tile (16..256, multiple of 16)
     int max_tiles;     // upper bound of the tile count
-    int s13_max;       // split-K bounds (device picks the actual split)
+    int s13_max;       // split-K bounds (the device picks the actual split)
     int s2_max;
     int grid;          // persistent CTAs
 };
@@ -76,18 +76,29 @@ struct FfnBuffers {
     const Tile* tiles;
     const int32_t* num_tiles;
     void* act;         // bf16 [R, I]
-    void* y;           // bf16 [R, H]
-    float* partials;   // fp32 split-K partials
-    int32_t* counters13;
-    int32_t* counters2;
+    void* y;           // bf16 [R, H]; written directly only when the w2 split is 1
+    float* partials;   // fp32 split-K partials (w13's, then reused by w2)
+    int32_t* splits;   // [2]: split counts the w13 and w2 kernels used
     int32_t* err;
 };
-// between_gemms: if not null, recorded on `st` after the w13 launch.
+// w13 (+ SwiGLU finalize when split) and w2.  between_gemms: if not null, recorded
+// on `st` after the w13 stage.  When the w2 split is > 1, y is left as partials:
+// the caller runs launch_combine (which reads them) or launch_reduce_y.
 cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, int I,
                                const FfnPlan& plan, cudaStream_t st,
                                cudaEvent_t between_gemms = nullptr);
 
-cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
-                           cudaStream_t st);
+// out[t] = sum_j w[t,j] * y[t*k+j]; y is taken from w2's partials (summed in slice
+// order, rounded to bf16) when *splits > 1, else from the bf16 y.  splits may be null.
+cudaError_t launch_combine(const void* y, const float* partials, const int32_t* splits,
+                           const float* weights, int T, int k, int H, void* out, cudaStream_t st);
+
+// act[p, f] = bf16(silu(sum_s gate_s) * sum_s up_s) when *splits > 1 (else no-op).
+cudaError_t launch_swiglu_finalize(const float* partials, const int32_t* splits, int R, int I,
+                                   void* act, cudaStream_t st);
+
+// y[r, h] = bf16(sum_s partial_s[r, h]) when *splits > 1 (else no-op).
+cudaError_t launch_reduce_y(const float* partials, const int32_t* splits, int R, int H, void* y,
+                            cudaStream_t st);
 
 }  // namespace moe

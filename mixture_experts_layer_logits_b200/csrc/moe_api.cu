@@ -65,8 +65,8 @@ bool combine_shape_ok(const moe_shape_t& s)
 }
 
 struct Layout {
-    size_t err, ids, weights, offsets, rows, tiles, num_tiles, counters13, counters2, chunks,
-        partials, act, y, total;
+    size_t err, ids, weights, offsets, rows, tiles, num_tiles, splits, chunks, partials, act, y,
+        total;
     FfnPlan plan;
     bool ffn;
 };
@@ -91,8 +91,7 @@ Layout layout_for(const moe_shape_t& s)
     L.rows = take(R * sizeof(int32_t));
     L.tiles = take((size_t)L.plan.max_tiles * sizeof(Tile));
     L.num_tiles = take(sizeof(int32_t));
-    L.counters13 = take((size_t)(I / 128) * L.plan.max_tiles * sizeof(int32_t));
-    L.counters2 = take((size_t)(H / 128) * L.plan.max_tiles * sizeof(int32_t));
+    L.splits = take(2 * sizeof(int32_t));
     const size_t n_chunks = (R + kChunkRows - 1) / kChunkRows;
     L.chunks = take(n_chunks * (size_t)s.E * sizeof(int32_t));
     if (L.ffn) {
@@ -140,9 +139,8 @@ PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
     a.tiles = at<Tile>(ws, L.tiles);
     a.num_tiles = at<int32_t>(ws, L.num_tiles);
     a.nt = L.plan.nt;
-    // both counter arrays are contiguous: one reset covers them
-    a.counters = at<int32_t>(ws, L.counters13);
-    a.n_counters = (int)((L.chunks - L.counters13) / sizeof(int32_t));
+    a.counters = nullptr;
+    a.n_counters = 0;
     a.chunk_counts = at<int32_t>(ws, L.chunks);
     (void)s;
     return a;
@@ -180,8 +178,7 @@ moe_status_t run_ffn(const void* x, const void* w13, const void* w2, const int32
     b.act = at<void>(ws, L.act);
     b.y = y;
     b.partials = at<float>(ws, L.partials);
-    b.counters13 = at<int32_t>(ws, L.counters13);
-    b.counters2 = at<int32_t>(ws, L.counters2);
+    b.splits = at<int32_t>(ws, L.splits);
     b.err = at<int32_t>(ws, L.err);
     FfnPlan plan = L.plan;
     plan.grid = device_sms();
@@ -247,7 +244,10 @@ moe_status_t moe_grouped_ffn(const moe_bf16_t* x, const moe_bf16_t* w13, const m
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     moe_status_t r = cuda_status(launch_build_tiles(expert_offsets, s.E, make_aux(ws, L, s), st));
     if (r != MOE_OK) return r;
-    return run_ffn(x, w13, w2, permuted_rows, s, y, ws, L, st);
+    r = run_ffn(x, w13, w2, permuted_rows, s, y, ws, L, st);
+    if (r != MOE_OK || L.plan.s2_max <= 1) return r;
+    return cuda_status(launch_reduce_y(at<float>(ws, L.partials), at<int32_t>(ws, L.splits),
+                                       s.T * s.top_k, s.H, y, st));
 }
 
 moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_shape_t s,
@@ -256,7 +256,7 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
     if (!y || !topk_weights || !out) return MOE_ERR_INVALID_ARG;
     if (!combine_shape_ok(s)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(y) || !aligned16(topk_weights) || !aligned16(out)) return MOE_ERR_MISALIGNED;
-    return cuda_status(launch_combine(y, topk_weights, s.T, s.top_k, s.H, out,
+    return cuda_status(launch_combine(y, nullptr, nullptr, topk_weights, s.T, s.top_k, s.H, out,
                                       static_cast<cudaStream_t>(stream)));
 }
 
@@ -292,7 +292,10 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
     if (r == MOE_OK) r = mark(1);
     if (r == MOE_OK) r = run_ffn(x, w13, w2, rows, s, y, ws, L, st, events ? events + 2 : nullptr);
     if (r == MOE_OK) r = mark(3);
-    if (r == MOE_OK) r = cuda_status(launch_combine(y, wts, s.T, s.top_k, s.H, out, st));
+    if (r == MOE_OK)
+        r = cuda_status(launch_combine(y, at<float>(ws, L.partials),
+                                       L.plan.s2_max > 1 ? at<int32_t>(ws, L.splits) + 1 : nullptr,
+                                       wts, s.T, s.top_k, s.H, out, st));
     if (r == MOE_OK) r = mark(4);
     return r;
 }
@@ -323,8 +326,9 @@ int moe_forward_kernel_count(moe_shape_t s)
 {
     if (!ffn_shape_ok(s)) return 0;
     const long R = (long)s.T * s.top_k;
-    // route(+permute) kernels, w13, w2, combine
-    return (R <= kSmallRows ? 1 : 4) + 2 + 1;
+    const Layout L = layout_for(s);
+    // route(+permute) kernels, w13, [SwiGLU finalize], w2, combine
+    return (R <= kSmallRows ? 1 : 4) + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
 }
 
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream)
