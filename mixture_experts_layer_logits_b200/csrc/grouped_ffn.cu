@@ -15,20 +15,25 @@
 // memory (fp32); MODE 0 keeps a gate and an up accumulator of equal shape so the
 // epilogue thread that owns feature f holds both halves of its SwiGLU pair.
 //
-// Warp roles (256 threads):
+// Warp roles (512 threads):
 //   warp 0      TMA producer: weight tiles [128 x 64] (and, MODE 1, the act tile
 //               [NT x 64]) with the 128-byte swizzle into a STAGES-deep ring.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
-//   warps 2-3   MODE 0 activation gather: 16-byte cp.async of x rows selected by
-//               permuted_rows[p] / k straight into the swizzled B tile (no
-//               permuted copy of x exists), then fence.proxy.async and an
-//               mbarrier arrival -- the writer-side proxy fence and barrier the
-//               FlashInfer PR #7368 page ("2. Hopper") requires before an async
-//               proxy reads generic-proxy stores.  The weight TMA for a stage is
-//               issued independently of the gather, so the two overlap (the
-//               BF16 ordering of the same section).
-//   warps 4-7   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//               32*(w%4) ..), SwiGLU / bf16 rounding / scatter, or split-K partials.
+//   warps 2-5   MODE 0 activation gather.  Gather warp g owns every stage whose
+//               sequence number is g mod 4: it issues 16-byte cp.async copies of
+//               the x rows selected by permuted_rows[p] / k straight into the
+//               swizzled B tile (no permuted copy of x exists), waits for them,
+//               then fence.proxy.async and one mbarrier arrival -- the writer-side
+//               proxy fence and barrier the FlashInfer PR #7368 page ("2. Hopper")
+//               requires before an async proxy reads generic-proxy stores.  The
+//               weight TMA of a stage is issued independently of its gather, so
+//               the two overlap (the BF16 ordering of the same section), and four
+//               stages can be in gather at once.
+//   warps 8-15  epilogue, two groups of four: tcgen05.ld of the accumulator
+//               (warp w reads TMEM lanes 32*(w%4) ..), group h owning the token
+//               columns [h*NT/2, (h+1)*NT/2); SwiGLU / bf16 rounding / scatter, or
+//               split-K partials.
+//   warps 6-7   idle.
 //
 // Split-K: when there are too few (tile, feature block) units to fill the GPU
 // (decode), each unit's K range is cut into S slices (S chosen on the device
@@ -57,7 +62,9 @@ namespace {
 constexpr int kBM = 128;        // weight rows per tile (MMA M)
 constexpr int kBK = 64;         // K elements per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 16;      // K per tcgen05.mma (bf16)
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;   // 16 warps, roles below
+constexpr int kGatherWarps = 4;  // warps 2..5
+constexpr int kEpiWarp0 = 8;     // warps 8..15: two epilogue groups of four
 constexpr int kATileBytes = kBM * kBK * 2;
 
 struct FfnArgs {
@@ -93,9 +100,12 @@ struct Cfg {
     static constexpr int kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64
                                    : kUsedCols <= 128 ? 128 : kUsedCols <= 256 ? 256 : 512;
     static constexpr uint32_t kTxBytes = kNA * kATileBytes + (MODE == 1 ? kBTileBytes : 0);
-    static constexpr int kGatherLag = (kStages - 1) < 3 ? (kStages - 1) : 3;
     // shared memory: 1 KB alignment slack + ring + barriers/aux
-    static constexpr int kAuxBytes = 1024 + 2 * NT * 4;
+    // Gather warps in use.  A waiter on a ring slot's mbarrier must never be more
+    // than one phase ahead of it (a parity wait cannot tell phase n from n - 2);
+    // gather warp g handles stages g, g + G, ..., so G <= kStages guarantees it.
+    static constexpr int kG = kGatherWarps < kStages ? kGatherWarps : kStages;
+    static constexpr int kAuxBytes = 1024 + kGatherWarps * NT * 4;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kAuxBytes;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N tile");
     static_assert(kStages >= 2, "pipeline depth");
@@ -128,11 +138,6 @@ __device__ __forceinline__ int split_count(const FfnArgs& a, int ntiles)
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
-__device__ __forceinline__ void named_bar_sync(int id, int n)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // bar.red.or over `n` threads: true in every thread if any thread passed true.
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
 {
@@ -148,7 +153,6 @@ __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
     return r != 0;
 }
 
-__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
 __device__ __forceinline__ void flag_error(const FfnArgs& a, Aux* aux)
 {
@@ -172,12 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&aux->full[s], MODE == 0 ? 1 + 64 : 1);
+            mbar_init(&aux->full[s], MODE == 0 ? 2 : 1);
             mbar_init(&aux->empty[s], 1);
         }
         for (int b = 0; b < C::kNBuf; ++b) {
             mbar_init(&aux->tfull[b], 1);
-            mbar_init(&aux->tempty[b], 4);
+            mbar_init(&aux->tempty[b], 8);
         }
         mbar_init(&aux->drain, 1);
         aux->abort = 0;
@@ -208,12 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.split_out = S;
     volatile int* abort_flag = &aux->abort;
 
-    // unit u -> (slice, tile, feature block); adjacent units share a weight block
+    // unit u -> (slice, feature block, tile), slice fastest: the feature blocks of a
+    // token tile run side by side (its x rows are re-read from L2, not HBM) and
+    // the tiles of one expert are neighbours (its weight blocks are shared in L2)
     auto decode = [&](int u, int& split, int& tile, int& fb) {
         split = u % S;
         const int rest = u / S;
-        tile = rest % ntiles;
-        fb = rest / ntiles;
+        fb = rest % a.fb_count;
+        tile = rest / a.fb_count;
     };
 
     if (warp == 0) {
@@ -320,29 +326,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             volatile int never = 0;
             if (!mbar_wait(&aux->drain, 0, &never, 500000000ull)) atomicExch(a.err, kDeviceErrorMagic);
         }
-    } else if (warp < 4) {
+    } else if (warp < 2 + kGatherWarps) {
         // ------------------------------------------------------------ gather (MODE 0)
-        if (MODE == 0) {
-            const int gt = threadIdx.x - 64;  // 0..63
-            constexpr int kLag = C::kGatherLag;
-            int ring_stage[4];
-            int issued = 0, arrived = 0;
-            int stage = 0;
-            uint32_t phase = 0;
+        if (MODE == 0 && warp - 2 < C::kG) {
+            constexpr int G = C::kG;
+            const int g = warp - 2;
+            int* my_off = tok_off + g * NT;
+            int q = 0;         // global stage sequence number (same as producer's)
+            int cur_tile = -1;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 int split, tile, fb;
                 decode(u, split, tile, fb);
-                const Tile t = a.tiles[tile];
                 const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
-                // each gather warp keeps its own copy of the tile's token offsets
-                int* my_off = tok_off + (warp - 2) * NT;
-                __syncwarp();  // previous unit's offsets are no longer read
-                for (int j = lane; j < t.rows; j += 32)
-                    my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
-                __syncwarp();
+                // first stage of this unit that this warp owns
+                int kt = kt0 + ((g - q % G) + G) % G;
+                const int q_unit0 = q;
+                q += kt1 - kt0;
+                if (kt >= kt1) continue;
+                const Tile t = a.tiles[tile];
+                if (tile != cur_tile) {
+                    __syncwarp();  // earlier copies' addresses are all issued
+                    for (int j = lane; j < t.rows; j += 32)
+                        my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
+                    __syncwarp();
+                    cur_tile = tile;
+                }
                 const int chunks = t.rows * 8;
-                for (int kt = kt0; kt < kt1; ++kt) {
+                for (; kt < kt1; kt += G) {
+                    const int qq = q_unit0 + (kt - kt0);
+                    const int stage = qq % C::kStages;
+                    const uint32_t phase = (uint32_t)((qq / C::kStages) & 1);
                     // warp-uniform decision, so no lane is left behind at __syncwarp
                     if (!__all_sync(0xffffffffu, mbar_wait(&aux->empty[stage], phase ^ 1u,
                                                            abort_flag))) {
@@ -353,30 +367,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bt =
                         smem_u32(ring + stage * C::kStageBytes + C::kNA * kATileBytes);
                     const __nv_bfloat16* src0 = a.x + kt * kBK;
-                    for (int q = gt; q < chunks; q += 64) {
-                        const int j = q >> 3, c = q & 7;
+                    for (int c8 = lane; c8 < chunks; c8 += 32) {
+                        const int j = c8 >> 3, c = c8 & 7;
                         cp_async_16(bt + j * 128 + ((c ^ (j & 7)) << 4), src0 + my_off[j] + c * 8);
                     }
                     cp_async_commit();
-                    ring_stage[issued & 3] = stage;
-                    ++issued;
-                    if (issued - arrived > kLag) {
-                        cp_async_wait<kLag>();
-                        fence_proxy_async_smem();
-                        while (issued - arrived > kLag) mbar_arrive(&aux->full[ring_stage[arrived++ & 3]]);
-                    }
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aux->full[stage]);
                 }
             }
             cp_async_wait<0>();
-            fence_proxy_async_smem();
-            while (arrived < issued) mbar_arrive(&aux->full[ring_stage[arrived++ & 3]]);
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        if (warp < kEpiWarp0) goto teardown;
+        const int grp = (warp - kEpiWarp0) >> 2;  // token-column half
         const int q = warp & 3;                 // TMEM lane quarter
         const int f_local = q * 32 + lane;      // feature inside the 128-row block
         const int pcols = (MODE == 0) ? 2 * a.I : a.H;
@@ -390,11 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
             const bool got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
             if (!got) flag_error(a, aux);
-            if (named_bar_or(1, 128, !got || *abort_flag)) break;  // same decision in all 4 warps
+            if (named_bar_or(1 + grp, 128, !got || *abort_flag)) break;  // same in all 4 warps
             tc_fence_after();
             const int f = fb * kBM + f_local;
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols);
-            for (int j0 = 0; j0 < t.rows; j0 += 16) {
+            const int jbeg = grp * (NT / 2), jend = min(t.rows, (grp + 1) * (NT / 2));
+            for (int j0 = jbeg; j0 < jend; j0 += 16) {
                 uint32_t g[16], v[16];
                 tmem_ld16(tacc + j0, g);
                 if (MODE == 0) tmem_ld16(tacc + NT + j0, v);
@@ -402,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int j = j0 + jj;
-                    if (j >= t.rows) break;
+                    if (j >= jend) break;
                     const int p = t.row_start + j;
                     const float gv = __uint_as_float(g[jj]);
                     if (S == 1) {
@@ -429,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+teardown:
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -524,12 +533,15 @@ FfnPlan plan_ffn(int T, int E, int k, int H, int I, int num_sms)
     while (nt < 256 && nt < T) nt *= 2;
     p.nt = nt;
     p.max_tiles = (int)((R + nt - 1) / nt + (E < R ? E : R));
-    // split-K only pays when even the smallest possible tile count leaves the GPU idle
+    // split-K only pays when even the smallest possible tile count leaves the GPU
+    // idle, and only for weight-streaming shapes: with >= 128 routed rows per
+    // expert on average the GEMMs are tensor-bound and a split only adds traffic
     const long min_units13 = ((R + nt - 1) / nt) * (I / kBM);
     const long min_units2 = ((R + nt - 1) / nt) * (H / kBM);
     const long target = 16L * num_sms;
-    p.s13_max = min_units13 >= target ? 1 : 8;
-    p.s2_max = min_units2 >= target ? 1 : 8;
+    const bool skinny = R < 128L * (E < R ? E : R);
+    p.s13_max = (skinny && min_units13 < target) ? 8 : 1;
+    p.s2_max = (skinny && min_units2 < target) ? 8 : 1;
     p.grid = num_sms;
     return p;
 }
