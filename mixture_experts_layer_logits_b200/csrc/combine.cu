@@ -22,7 +22,12 @@ namespace moe {
 
 namespace {
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u with the same fast exponential and reciprocal as the GEMM epilogue
+// (the product is rounded to bf16).
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    return g * __frcp_rn(1.0f + __expf(-g)) * u;
+}
 
 __device__ __forceinline__ void add4(float (&a)[8], int o, float4 v)
 {
@@ -47,6 +52,7 @@ __global__ void __launch_bounds__(256)
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 8
     for (int j = 0; j < k; ++j) {
         const long r = (long)t * k + j;
         const float wj = __ldg(w + r);
@@ -63,7 +69,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
             for (int i = 0; i < 8; ++i) yv[i] = __bfloat162float(__float2bfloat16_rn(s8[i]));
         } else {
-            const uint4 v = __ldcs(y + r * H8 + h8);  // read once: stream
+            const uint4 v = __ldcs(y + r * H8 + h8);  // read once: stream (the j loop is
+                                                     // unrolled so the k loads overlap)
             const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {

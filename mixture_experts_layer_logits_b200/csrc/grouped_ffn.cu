@@ -63,8 +63,9 @@ constexpr int kBM = 128;        // weight rows per tile (MMA M)
 constexpr int kBK = 64;         // K elements per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 16;      // K per tcgen05.mma (bf16)
 constexpr int kThreads = 512;   // 16 warps, roles below
-constexpr int kGatherWarps = 4;  // warps 2..5
+constexpr int kGatherWarps = 6;  // warps 2..7
 constexpr int kEpiWarp0 = 8;     // warps 8..15: two epilogue groups of four
+constexpr int kPrefetch = 4;     // weight K-tiles brought to L2 ahead of their TMA
 constexpr int kATileBytes = kBM * kBK * 2;
 
 struct FfnArgs {
@@ -78,7 +79,7 @@ struct FfnArgs {
     int32_t* err;
     int k, H, I, R;
     int num_kt;               // K / 64
-    int fb_count;             // feature blocks of 128
+    int fb_count;             // MODE 0: gate/up block pairs (I / 128); MODE 1: 256-row blocks
     int s_max;                // split-K upper bound
     int max_tiles;
     int min_kt_per_split;
@@ -87,13 +88,13 @@ struct FfnArgs {
 
 template <int MODE, int NT>
 struct Cfg {
-    static constexpr int kNA = (MODE == 0) ? 2 : 1;               // A tiles per stage
+    static constexpr int kNA = 2;                                  // A tiles per stage
     static constexpr int kBTileBytes = NT * kBK * 2;
     static constexpr int kStageBytes = kNA * kATileBytes + kBTileBytes;
     static constexpr int kBudget = 220 * 1024;
     static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kAccCols = (MODE == 0) ? 2 * NT : NT;    // per accumulator buffer
+    static constexpr int kAccCols = 2 * NT;                        // per accumulator buffer
     static constexpr int kNBufRaw = 512 / kAccCols;                // accumulators in flight
     static constexpr int kNBuf = kNBufRaw > 8 ? 8 : kNBufRaw;
     static constexpr int kUsedCols = kAccCols * kNBuf;
@@ -101,10 +102,12 @@ struct Cfg {
                                    : kUsedCols <= 128 ? 128 : kUsedCols <= 256 ? 256 : 512;
     static constexpr uint32_t kTxBytes = kNA * kATileBytes + (MODE == 1 ? kBTileBytes : 0);
     // shared memory: 1 KB alignment slack + ring + barriers/aux
-    // Gather warps in use.  A waiter on a ring slot's mbarrier must never be more
-    // than one phase ahead of it (a parity wait cannot tell phase n from n - 2);
-    // gather warp g handles stages g, g + G, ..., so G <= kStages guarantees it.
+    // Gather groups.  A waiter on a ring slot's mbarrier must never be more than one
+    // phase ahead of it (a parity wait cannot tell phase n from n - 2); group g
+    // handles stages g, g + G, ..., so G <= kStages guarantees it.  The W warps of
+    // a group split the rows of its stages.
     static constexpr int kG = kGatherWarps < kStages ? kGatherWarps : kStages;
+    static constexpr int kW = kGatherWarps / kG;
     static constexpr int kAuxBytes = 1024 + kGatherWarps * NT * 4;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kAuxBytes;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N tile");
@@ -136,7 +139,13 @@ __device__ __forceinline__ int split_count(const FfnArgs& a, int ntiles)
     return max(s, 1);
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u = g * u / (1 + e^-g).  The result is rounded to bf16 (8-bit
+// significand), so the fast exponential and reciprocal (a few ulp of fp32) are
+// far inside that rounding; for g -> -inf the reciprocal of inf is 0.
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    return g * __frcp_rn(1.0f + __expf(-g)) * u;
+}
 
 // bar.red.or over `n` threads: true in every thread if any thread passed true.
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
@@ -176,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&aux->full[s], MODE == 0 ? 2 : 1);
+            mbar_init(&aux->full[s], MODE == 0 ? 1 + C::kW : 1);
             mbar_init(&aux->empty[s], 1);
         }
         for (int b = 0; b < C::kNBuf; ++b) {
@@ -225,8 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            // decode streams each weight block once; larger batches share a block
+            // between the tiles of one expert, so leave those at normal priority
             const uint64_t pol = a.weights_evict_first ? l2_policy_evict_first()
-                                                       : l2_policy_evict_last();
+                                                       : l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
             int issued[16];
@@ -251,10 +262,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(st + kATileBytes, &tm_w, &aux->full[stage], kt * kBK, row + a.I,
                                     pol);
                     } else {
-                        const int row = t.expert * a.H + fb * kBM;
+                        // two consecutive 128-row blocks of w2[e]; when H is an odd number
+                        // of 128-row blocks the second block of the last pair belongs to
+                        // the next expert (or lies past the tensor and is zero-filled)
+                        // and its accumulator is never stored
+                        const int row = t.expert * a.H + fb * 2 * kBM;
                         tma_load_2d(st, &tm_w, &aux->full[stage], kt * kBK, row, pol);
-                        tma_load_2d_nohint(st + kATileBytes, &tm_act, &aux->full[stage], kt * kBK,
-                                           t.row_start);
+                        tma_load_2d(st + kATileBytes, &tm_w, &aux->full[stage], kt * kBK,
+                                    row + kBM, pol);
+                        tma_load_2d_nohint(st + 2 * kATileBytes, &tm_act, &aux->full[stage],
+                                           kt * kBK, t.row_start);
+                    }
+                    // weight tiles kPrefetch stages ahead go to L2 now, so the TMA that
+                    // needs them later finds them there (the ring holds only a few stages)
+                    // (weight-streaming shapes read each block once: nothing to gain there)
+                    if (!a.weights_evict_first && kt + kPrefetch < kt1) {
+                        const int row = MODE == 0 ? t.expert * 2 * a.I + fb * kBM
+                                                  : t.expert * a.H + fb * 2 * kBM;
+                        const int row1 = MODE == 0 ? row + a.I : row + kBM;
+                        tma_prefetch_l2_2d(&tm_w, (kt + kPrefetch) * kBK, row);
+                        tma_prefetch_l2_2d(&tm_w, (kt + kPrefetch) * kBK, row1);
                     }
                     issued[stage] += 1;
                     if (++stage == C::kStages) {
@@ -309,9 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t acc = (kt > kt0 || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
                         umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
-                        if (MODE == 0)
-                            umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
-                                      idesc, acc);
+                        umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
+                                  idesc, acc);
                     }
                     umma_commit(&aux->empty[stage]);  // frees the smem stage when read
                     if (++stage == C::kStages) {
@@ -328,10 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 2 + kGatherWarps) {
         // ------------------------------------------------------------ gather (MODE 0)
-        if (MODE == 0 && warp - 2 < C::kG) {
-            constexpr int G = C::kG;
-            const int g = warp - 2;
-            int* my_off = tok_off + g * NT;
+        if (MODE == 0 && warp - 2 < C::kG * C::kW) {
+            constexpr int G = C::kG, W = C::kW;
+            const int g = (warp - 2) / W, wi = (warp - 2) % W;
+            int* my_off = tok_off + (warp - 2) * NT;
+            const uint64_t x_policy = l2_policy_evict_last();  // x rows are re-read per block
             int q = 0;         // global stage sequence number (same as producer's)
             int cur_tile = -1;
             bool ok = true;
@@ -367,9 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bt =
                         smem_u32(ring + stage * C::kStageBytes + C::kNA * kATileBytes);
                     const __nv_bfloat16* src0 = a.x + kt * kBK;
-                    for (int c8 = lane; c8 < chunks; c8 += 32) {
+                    for (int c8 = lane + 32 * wi; c8 < chunks; c8 += 32 * W) {
                         const int j = c8 >> 3, c = c8 & 7;
-                        cp_async_16(bt + j * 128 + ((c ^ (j & 7)) << 4), src0 + my_off[j] + c * 8);
+                        cp_async_16_hint(bt + j * 128 + ((c ^ (j & 7)) << 4),
+                                         src0 + my_off[j] + c * 8, x_policy);
                     }
                     cp_async_commit();
                     cp_async_wait<0>();
@@ -399,13 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!got) flag_error(a, aux);
             if (named_bar_or(1 + grp, 128, !got || *abort_flag)) break;  // same in all 4 warps
             tc_fence_after();
-            const int f = fb * kBM + f_local;
+            // MODE 0: feature f of the gate block (accumulator 0) and of the up block
+            // (accumulator 1); MODE 1: output features f and f + 128
+            const int f = (MODE == 0 ? fb * kBM : fb * 2 * kBM) + f_local;
+            const bool f1_ok = MODE == 0 || f + kBM < a.H;
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols);
             const int jbeg = grp * (NT / 2), jend = min(t.rows, (grp + 1) * (NT / 2));
             for (int j0 = jbeg; j0 < jend; j0 += 16) {
                 uint32_t g[16], v[16];
                 tmem_ld16(tacc + j0, g);
-                if (MODE == 0) tmem_ld16(tacc + NT + j0, v);
+                tmem_ld16(tacc + NT + j0, v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
@@ -420,6 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else {
                             const int r = a.permuted_rows[p];
                             a.out[(size_t)r * ocols + f] = __float2bfloat16_rn(gv);
+                            if (f1_ok)
+                                a.out[(size_t)r * ocols + f + kBM] =
+                                    __float2bfloat16_rn(__uint_as_float(v[jj]));
                         }
                     } else if (MODE == 0) {
                         float* prow = a.partials + ((size_t)split * a.R + p) * pcols;
@@ -427,7 +461,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         prow[a.I + f] = __uint_as_float(v[jj]);
                     } else {
                         const int r = a.permuted_rows[p];
-                        a.partials[((size_t)split * a.R + r) * pcols + f] = gv;
+                        float* prow = a.partials + ((size_t)split * a.R + r) * pcols;
+                        prow[f] = gv;
+                        if (f1_ok) prow[f + kBM] = __uint_as_float(v[jj]);
                     }
                 }
             }
@@ -592,7 +628,7 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
     a.out = static_cast<__nv_bfloat16*>(b.y);
     a.split_out = b.splits + 1;
     a.num_kt = I / kBK;
-    a.fb_count = H / kBM;
+    a.fb_count = (H / kBM + 1) / 2;
     a.s_max = plan.s2_max;
     return launch_nt<1>(plan.nt, tw2, tact, a, plan.grid, st);
 }

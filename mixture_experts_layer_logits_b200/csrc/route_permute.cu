@@ -133,19 +133,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sums, int& total
     return prefix + incl - v;
 }
 
-// Thread e (< E) owns expert e with `count` rows at permuted offset `off`;
-// writes its ceil(count / nt) tiles.  Also zeroes the split-K counters.
+// Thread e (< E) owns expert e with `count` rows at permuted offset `off` and
+// writes its tiles: as few as ceil(count / nt) allows, of near-equal size rounded
+// to the MMA's 16-column granule (so no tile is a short tail that streams a whole
+// weight block for a few rows), the last one taking the remainder.
+// Also zeroes the split-K counters.
 __device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int count, int off,
                                                       const PermuteAux& aux, int* sums)
 {
-    const int n = owns ? (count + aux.nt - 1) / aux.nt : 0;
+    int n = 0, q = aux.nt;
+    if (owns && count > 0) {
+        const int n0 = (count + aux.nt - 1) / aux.nt;
+        const int even = (count + n0 - 1) / n0;
+        q = min(aux.nt, (even + 15) & ~15);
+        n = (count + q - 1) / q;
+    }
     int total;
     const int start = block_exclusive_scan(n, sums, total);
     for (int i = 0; i < n; ++i) {
         Tile t;
         t.expert = e;
-        t.row_start = off + i * aux.nt;
-        t.rows = min(aux.nt, count - i * aux.nt);
+        t.row_start = off + i * q;
+        t.rows = min(q, count - i * q);
         t.pad = 0;
         aux.tiles[start + i] = t;
     }
