@@ -75,6 +75,27 @@ def get_workload(spec):
                      dup_frac=float(kv.get("dup", 0.0)))
 
 
+def rank_seed(seed, rank):
+    """Seed of one rank's tokens (logits, x); the weights use `seed` on every rank."""
+    return seed + rank
+
+
+def max_over_ranks(value, pg=None, device="cpu"):
+    """The slowest rank's figure (all ranks take part, same call order everywhere)."""
+    if pg is None:
+        return value
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, tokens_per_rank, ms_slowest):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_slowest / 1e3)
+
+
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
@@ -294,7 +315,7 @@ def routing_bench(args, w, rank, world, local, dev, pg):
 
     T, E, k = w.T, w.E, w.k
     R = T * k
-    logits = wl.make_logits(w, seed=args.seed + rank, device=dev)
+    logits = wl.make_logits(w, seed=rank_seed(args.seed, rank), device=dev)
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
     wts = torch.empty(T, k, dtype=torch.float32, device=dev)
     off = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -318,12 +339,8 @@ def routing_bench(args, w, rank, world, local, dev, pg):
         if pg:
             pg.barrier()
 
-    def max_over_ranks(v):
-        if not pg:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(v):
+        return max_over_ranks(v, pg, dev)
 
     W = max(args.warmup, 3)
     for _ in range(W):
@@ -339,9 +356,9 @@ def routing_bench(args, w, rank, world, local, dev, pg):
             step(ev[i])
         barrier()
         t_wall = time.perf_counter() - t_wall
-    ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
-    route_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
-    perm_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    ms = slowest(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
+    route_ms = slowest(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    perm_ms = slowest(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
 
     # e2e: logits from pinned host memory in, the four outputs back out
     logits_h = logits.cpu().pin_memory()
@@ -359,7 +376,7 @@ def routing_bench(args, w, rank, world, local, dev, pg):
             h.copy_(d, non_blocking=True)
         eev[i][1].record(stream)
     barrier()
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in eev))
+    e2e_ms = slowest(statistics.mean(a.elapsed_time(b) for a, b in eev))
 
     peaks, peak_kind = load_peaks()
     route_bytes = T * E * 4 + R * 8
@@ -386,7 +403,7 @@ def routing_bench(args, w, rank, world, local, dev, pg):
         all_bytes = route_bytes + perm_bytes
         launches = 1 + (1 if R <= 4096 else 3)
         line = {
-            "metric": metric_name(w), "value": round(world * T / (ms / 1e3), 2),
+            "metric": metric_name(w), "value": round(weak_scaling_value(world, T, ms), 2),
             "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
@@ -453,8 +470,8 @@ def main(argv=None):
     T, E, k, H, I = w.T, w.E, w.k, w.H, w.I
     R = T * k
     # this rank's tokens; weights are the same on every rank
-    logits = wl.make_logits(w, seed=args.seed + rank, device=dev)
-    x = wl.make_x(w, seed=args.seed + rank, device=dev)
+    logits = wl.make_logits(w, seed=rank_seed(args.seed, rank), device=dev)
+    x = wl.make_x(w, seed=rank_seed(args.seed, rank), device=dev)
     w13, w2 = wl.make_weights(w, seed=args.seed, device=dev)
     ws = moe.workspace(T, E, k, H, I, device=dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
@@ -474,12 +491,8 @@ def main(argv=None):
         if pg:
             pg.barrier()
 
-    def max_over_ranks(v):
-        if not pg:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(v):
+        return max_over_ranks(v, pg, dev)
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
@@ -504,7 +517,7 @@ def main(argv=None):
         barrier()
         t_wall = time.perf_counter() - t_wall
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = max_over_ranks(statistics.mean(step_ms))
+    ms = slowest(statistics.mean(step_ms))
     if moe.moe_device_status(ws) != moe.MOE_OK:
         raise SystemExit("device error during the timed steps")
 
@@ -523,7 +536,7 @@ def main(argv=None):
     names = ["route_permute", "w13", "w2", "combine"]
     stage_ms = {n: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(KB))
                 for j, n in enumerate(names)}
-    stage_ms = {n: max_over_ranks(v) for n, v in stage_ms.items()}
+    stage_ms = {n: slowest(v) for n, v in stage_ms.items()}
 
     # ---- pass C: end to end from pinned host memory
     KC = min(K, 200)
@@ -542,7 +555,7 @@ def main(argv=None):
         out_h.copy_(out, non_blocking=True)
         eev[i][1].record(stream)
     barrier()
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in eev))
+    e2e_ms = slowest(statistics.mean(a.elapsed_time(b) for a, b in eev))
     h2d = x_h.numel() * x_h.element_size() + logits_h.numel() * logits_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 
@@ -570,7 +583,7 @@ def main(argv=None):
         launches = moe.moe_forward_kernel_count(T, E, k, H, I)
         line = {
             "metric": metric_name(w),
-            "value": round(world * T / (ms / 1e3), 2),
+            "value": round(weak_scaling_value(world, T, ms), 2),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": K,
