@@ -66,6 +66,8 @@ constexpr int kThreads = 512;   // 16 warps, roles below
 constexpr int kGatherWarps = 6;  // warps 2..7
 constexpr int kEpiWarp0 = 8;     // warps 8..15: two epilogue groups of four
 constexpr int kPrefetch = 4;     // weight K-tiles brought to L2 ahead of their TMA
+constexpr int kStageRows = 8;    // token rows per epilogue staging buffer
+constexpr int kStageRowBytes = 512;  // one token row: 256 bf16 outputs
 constexpr int kATileBytes = kBM * kBK * 2;
 
 struct FfnArgs {
@@ -91,8 +93,12 @@ struct Cfg {
     static constexpr int kNA = 2;                                  // A tiles per stage
     static constexpr int kBTileBytes = NT * kBK * 2;
     static constexpr int kStageBytes = kNA * kATileBytes + kBTileBytes;
-    static constexpr int kBudget = 220 * 1024;
-    static constexpr int kStagesRaw = kBudget / kStageBytes;
+    // shared memory: 1 KB alignment slack | ring | epilogue staging | Aux | token offsets
+    static constexpr int kMaxSmem = 232448;  // 227 KB per CTA
+    static constexpr int kAuxBytes = 1024 + kGatherWarps * NT * 4;
+    static constexpr int kStagingBytes = 2 * 2 * kStageRows * kStageRowBytes;  // 2 groups x 2 bufs
+    static constexpr int kStagesRaw =
+        (kMaxSmem - 1024 - kAuxBytes - kStagingBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kAccCols = 2 * NT;                        // per accumulator buffer
     static constexpr int kNBufRaw = 512 / kAccCols;                // accumulators in flight
@@ -108,8 +114,7 @@ struct Cfg {
     // a group split the rows of its stages.
     static constexpr int kG = kGatherWarps < kStages ? kGatherWarps : kStages;
     static constexpr int kW = kGatherWarps / kG;
-    static constexpr int kAuxBytes = 1024 + kGatherWarps * NT * 4;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kAuxBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kStagingBytes + kAuxBytes;
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N tile");
     static_assert(kStages >= 2, "pipeline depth");
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
@@ -147,6 +152,11 @@ __device__ __forceinline__ float silu_mul(float g, float u)
     return g * __frcp_rn(1.0f + __expf(-g)) * u;
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // bar.red.or over `n` threads: true in every thread if any thread passed true.
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
 {
@@ -178,7 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    Aux* aux = reinterpret_cast<Aux*>(ring + C::kStages * C::kStageBytes);
+    uint8_t* staging = ring + C::kStages * C::kStageBytes;
+    Aux* aux = reinterpret_cast<Aux*>(staging + C::kStagingBytes);
     int* tok_off = reinterpret_cast<int*>(aux + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -221,14 +232,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.split_out = S;
     volatile int* abort_flag = &aux->abort;
 
-    // unit u -> (slice, feature block, tile), slice fastest: the feature blocks of a
-    // token tile run side by side (its x rows are re-read from L2, not HBM) and
-    // the tiles of one expert are neighbours (its weight blocks are shared in L2)
+    // unit u -> (slice, tile, feature block), expert-grouped: the units of expert e
+    // occupy [fb_count * first_e, fb_count * (first_e + count_e)), feature block
+    // major and tile minor, so the tiles that share a weight block are adjacent
+    // (they run at the same time on neighbouring CTAs and share it in L2), and the
+    // feature blocks of a tile run close together (its x rows stay in L2).  Since
+    // fb_count * first_e <= rest < fb_count * first_{e+1}, tile rest / fb_count
+    // belongs to expert e and carries first_e and count_e.  Slice fastest.
     auto decode = [&](int u, int& split, int& tile, int& fb) {
         split = u % S;
         const int rest = u / S;
-        fb = rest % a.fb_count;
-        tile = rest / a.fb_count;
+        const Tile& probe = a.tiles[rest / a.fb_count];
+        const int local = rest - a.fb_count * probe.first;
+        fb = local / probe.count;
+        tile = probe.first + local % probe.count;
     };
 
     if (warp == 0) {
@@ -416,6 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f_local = q * 32 + lane;      // feature inside the 128-row block
         const int pcols = (MODE == 0) ? 2 * a.I : a.H;
         const int ocols = (MODE == 0) ? a.I : a.H;
+        int chunk = 0;  // staging chunks issued by this group (buffer parity)
         int lu = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++lu) {
             int split, tile, fb;
@@ -433,6 +451,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool f1_ok = MODE == 0 || f + kBM < a.H;
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols);
             const int jbeg = grp * (NT / 2), jend = min(t.rows, (grp + 1) * (NT / 2));
+            if (S == 1) {
+                // Stage 8 token rows at a time in shared memory ([row][256 outputs] bf16),
+                // then the group's 128 threads copy them out with 16-byte loads and
+                // stores, each output row written whole and coalesced (256 B of act in
+                // MODE 0, up to 512 B of y in MODE 1).  Two buffers per group: one
+                // barrier per chunk separates a buffer's readers from its next writers.
+                const int row_bytes = MODE == 0 ? 2 * kBM : ((fb * 2 + 1) * kBM < a.H ? 4 * kBM : 2 * kBM);
+                const int vec_per_row = row_bytes / 16;
+                for (int j0 = jbeg; j0 < jend; j0 += kStageRows) {
+                    uint32_t g[8], v[8];
+                    tmem_ld8(tacc + j0, g);
+                    tmem_ld8(tacc + NT + j0, v);
+                    tmem_ld_wait();
+                    if (j0 + kStageRows >= jend) {  // accumulator drained: let the MMA go on
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&aux->tempty[b]);
+                    }
+                    uint8_t* buf = staging + (grp * 2 + (chunk & 1)) * (kStageRows * kStageRowBytes);
+#pragma unroll
+                    for (int jj = 0; jj < kStageRows; ++jj) {
+                        __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(buf + jj * kStageRowBytes);
+                        if (MODE == 0) {
+                            row[f_local] = __float2bfloat16_rn(
+                                silu_mul(__uint_as_float(g[jj]), __uint_as_float(v[jj])));
+                        } else {
+                            row[f_local] = __float2bfloat16_rn(__uint_as_float(g[jj]));
+                            row[kBM + f_local] = __float2bfloat16_rn(__uint_as_float(v[jj]));
+                        }
+                    }
+                    named_bar_sync(1 + grp, 128);  // staged; the other buffer is free again
+                    const int n = min(kStageRows, jend - j0);
+                    const int gt = (warp & 3) * 32 + lane;  // 0..127 within the group
+                    for (int i = gt; i < n * vec_per_row; i += 128) {
+                        const int jj = i / vec_per_row, c = i % vec_per_row;
+                        const int p = t.row_start + j0 + jj;
+                        const uint4 val = *reinterpret_cast<const uint4*>(buf + jj * kStageRowBytes + c * 16);
+                        __nv_bfloat16* dst = MODE == 0
+                            ? a.out + (size_t)p * ocols + fb * kBM
+                            : a.out + (size_t)a.permuted_rows[p] * ocols + fb * 2 * kBM;
+                        *reinterpret_cast<uint4*>(dst + c * 8) = val;
+                    }
+                    ++chunk;
+                }
+                if (jbeg >= jend) {  // this group had no columns of the unit
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aux->tempty[b]);
+                }
+                continue;
+            }
             for (int j0 = jbeg; j0 < jend; j0 += 16) {
                 uint32_t g[16], v[16];
                 tmem_ld16(tacc + j0, g);
@@ -444,18 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j >= jend) break;
                     const int p = t.row_start + j;
                     const float gv = __uint_as_float(g[jj]);
-                    if (S == 1) {
-                        if (MODE == 0) {
-                            a.out[(size_t)p * ocols + f] =
-                                __float2bfloat16_rn(silu_mul(gv, __uint_as_float(v[jj])));
-                        } else {
-                            const int r = a.permuted_rows[p];
-                            a.out[(size_t)r * ocols + f] = __float2bfloat16_rn(gv);
-                            if (f1_ok)
-                                a.out[(size_t)r * ocols + f + kBM] =
-                                    __float2bfloat16_rn(__uint_as_float(v[jj]));
-                        }
-                    } else if (MODE == 0) {
+                    if (MODE == 0) {
                         float* prow = a.partials + ((size_t)split * a.R + p) * pcols;
                         prow[f] = gv;
                         prow[a.I + f] = __uint_as_float(v[jj]);

@@ -14,12 +14,15 @@ namespace moe {
 constexpr int32_t kDeviceErrorMagic = 0x4D4F4554;
 
 // One tile of the grouped GEMMs: `rows` (1..NT) consecutive permuted rows of one
-// expert, starting at permuted position `row_start`.
+// expert, starting at permuted position `row_start`.  `first` is the index of the
+// expert's first tile and `count` its number of tiles.
 struct Tile {
     int expert;
     int row_start;
     int rows;
-    int pad;
+    int first;
+    int count;
+    int pad[3];
 };
 
 // Everything the route/permute kernels write besides the user-visible outputs.

@@ -155,7 +155,9 @@ __device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int coun
         t.expert = e;
         t.row_start = off + i * q;
         t.rows = min(q, count - i * q);
-        t.pad = 0;
+        t.first = start;
+        t.count = n;
+        t.pad[0] = t.pad[1] = t.pad[2] = 0;
         aux.tiles[start + i] = t;
     }
     if (threadIdx.x == 0) *aux.num_tiles = total;
