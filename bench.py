@@ -351,9 +351,11 @@ def routing_bench(args, w, rank, world, local, dev, pg):
     barrier()
     with ClockSampler(local) as clocks:
         t_wall = time.perf_counter()
+        torch.cuda.nvtx.range_push("timed")
         for i in range(K):
             flush.zero_()
             step(ev[i])
+        torch.cuda.nvtx.range_pop()
         barrier()
         t_wall = time.perf_counter() - t_wall
     ms = slowest(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
@@ -509,11 +511,13 @@ def main(argv=None):
     barrier()
     with ClockSampler(local) as clocks:
         t_wall = time.perf_counter()
+        torch.cuda.nvtx.range_push("timed")  # lets a profiler select the timed steps
         for i in range(K):
             flush.zero_()
             ev[i][0].record(stream)
             fwd()
             ev[i][1].record(stream)
+        torch.cuda.nvtx.range_pop()
         barrier()
         t_wall = time.perf_counter() - t_wall
     step_ms = [a.elapsed_time(b) for a, b in ev]

@@ -3,14 +3,14 @@
 //   combine          out[t] = sum_{j=0..k-1} w[t, j] * y[t*k + j], fp32, j ascending,
 //                    rounded once to bf16 (the fixed-order fp32 merge principle of the
 //                    "FP32 partials" section of the FlashInfer PR #5586 page, applied
-//                    to the top-k combine).  When the w2 GEMM ran split-K, y[r] is
-//                    first rebuilt as bf16(sum_s partial_s[r]) in slice order, so the
-//                    result is the same as combining a materialised y.
+//                    to the top-k combine).
 //   swiglu finalize  act[p, f] = bf16(silu(sum_s gate_s) * sum_s up_s) for a split w13.
-//   reduce y         y[r, h] = bf16(sum_s partial_s[r, h]) for a split w2 whose y is
-//                    wanted on its own (moe_grouped_ffn).
+//   reduce y         y[r, h] = bf16(sum_s partial_s[r, h]) for a split w2 (before the
+//                    combine, or for moe_grouped_ffn's y).
 //
-// Each thread moves 16-byte vectors; the split count is read on the device.
+// Each thread moves 16-byte vectors and issues all of its loads before using any
+// (these kernels are short and latency-bound at decode sizes); the split count
+// is read on the device.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -29,58 +29,44 @@ __device__ __forceinline__ float silu_mul(float g, float u)
     return g * __frcp_rn(1.0f + __expf(-g)) * u;
 }
 
-__device__ __forceinline__ void add4(float (&a)[8], int o, float4 v)
-{
-    a[o] += v.x;
-    a[o + 1] += v.y;
-    a[o + 2] += v.z;
-    a[o + 3] += v.w;
-}
+constexpr int kMaxK = 16;
+constexpr int kMaxSplits = 8;
 
+// One thread per (token, 8 hidden elements): the k rows are all loaded before
+// any is used, so a thread keeps up to 16 loads in flight.
 __global__ void __launch_bounds__(256)
-    combine_kernel(const uint4* __restrict__ y, const float4* __restrict__ partials,
-                   const int32_t* __restrict__ splits, const float* __restrict__ w, int T, int k,
-                   int H8, uint4* __restrict__ out)
+    combine_kernel(const uint4* __restrict__ y, const float* __restrict__ w, int T, int k, int H8,
+                   uint4* __restrict__ out)
 {
     pdl_wait();
     pdl_launch_dependents();
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long)T * H8) return;
-    const int S = splits ? *splits : 1;
     const int t = (int)(idx / H8), h8 = (int)(idx % H8);
-    const long R = (long)T * k;
+    uint4 v[kMaxK];
+    float wj[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        if (j < k) {
+            const long r = (long)t * k + j;
+            v[j] = __ldcs(y + r * H8 + h8);  // read once: stream
+            wj[j] = __ldg(w + r);
+        }
+    }
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-        const long r = (long)t * k + j;
-        const float wj = __ldg(w + r);
-        float yv[8];
-        if (S > 1) {
-            float s8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) s8[i] = 0.f;
-            for (int s = 0; s < S; ++s) {  // slice order
-                const float4* pr = partials + ((size_t)s * R + r) * (H8 * 2) + h8 * 2;
-                add4(s8, 0, __ldcs(pr));
-                add4(s8, 4, __ldcs(pr + 1));
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) yv[i] = __bfloat162float(__float2bfloat16_rn(s8[i]));
-        } else {
-            const uint4 v = __ldcs(y + r * H8 + h8);  // read once: stream (the j loop is
-                                                     // unrolled so the k loads overlap)
-            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+    for (int j = 0; j < kMaxK; ++j) {
+        if (j < k) {  // j ascending: the fixed summation order
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float2 f = __bfloat1622float2(p[i]);
-                yv[2 * i] = f.x;
-                yv[2 * i + 1] = f.y;
+                acc[2 * i] = fmaf(wj[j], f.x, acc[2 * i]);
+                acc[2 * i + 1] = fmaf(wj[j], f.y, acc[2 * i + 1]);
             }
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, yv[i], acc[i]);
     }
     uint4 o;
     __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -102,12 +88,22 @@ __global__ void __launch_bounds__(256)
     if (idx >= (long)R * I4) return;
     const long p = idx / I4;
     const int f4 = (int)(idx % I4);
+    float4 pa[kMaxSplits], pb[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {  // every slice's loads in flight at once
+        if (s < S) {
+            const float4* row = partials + ((size_t)s * R + p) * (2 * I4);
+            pa[s] = __ldcs(row + f4);
+            pb[s] = __ldcs(row + I4 + f4);
+        }
+    }
     float g[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < S; ++s) {
-        const float4* row = partials + ((size_t)s * R + p) * (2 * I4);
-        const float4 a = __ldcs(row + f4), b = __ldcs(row + I4 + f4);
-        g[0] += a.x; g[1] += a.y; g[2] += a.z; g[3] += a.w;
-        u[0] += b.x; u[1] += b.y; u[2] += b.z; u[3] += b.w;
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {  // slice order
+        if (s < S) {
+            g[0] += pa[s].x; g[1] += pa[s].y; g[2] += pa[s].z; g[3] += pa[s].w;
+            u[0] += pb[s].x; u[1] += pb[s].y; u[2] += pb[s].z; u[3] += pb[s].w;
+        }
     }
     uint2 o;
     __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -127,10 +123,16 @@ __global__ void __launch_bounds__(256)
     if (S <= 1) return;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long)R * H4) return;
+    float4 pv[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+        if (s < S) pv[s] = __ldcs(partials + (size_t)s * R * H4 + idx);
     float a[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < S; ++s) {
-        const float4 v = __ldcs(partials + (size_t)s * R * H4 + idx);
-        a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {  // slice order
+        if (s < S) {
+            a[0] += pv[s].x; a[1] += pv[s].y; a[2] += pv[s].z; a[3] += pv[s].w;
+        }
     }
     uint2 o;
     __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -156,13 +158,12 @@ cudaError_t launch_1d(Kern kern, long n, cudaStream_t st, Args... args)
 
 }  // namespace
 
-cudaError_t launch_combine(const void* y, const float* partials, const int32_t* splits,
-                           const float* weights, int T, int k, int H, void* out, cudaStream_t st)
+cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
+                           cudaStream_t st)
 {
     const int H8 = H / 8;
-    return launch_1d(combine_kernel, (long)T * H8, st, static_cast<const uint4*>(y),
-                     reinterpret_cast<const float4*>(partials), splits, weights, T, k, H8,
-                     static_cast<uint4*>(out));
+    return launch_1d(combine_kernel, (long)T * H8, st, static_cast<const uint4*>(y), weights, T, k,
+                     H8, static_cast<uint4*>(out));
 }
 
 cudaError_t launch_swiglu_finalize(const float* partials, const int32_t* splits, int R, int I,

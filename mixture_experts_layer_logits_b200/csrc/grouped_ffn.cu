@@ -688,7 +688,9 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
     a.num_kt = I / kBK;
     a.fb_count = (H / kBM + 1) / 2;
     a.s_max = plan.s2_max;
-    return launch_nt<1>(plan.nt, tw2, tact, a, plan.grid, st);
+    err = launch_nt<1>(plan.nt, tw2, tact, a, plan.grid, st);
+    if (err != cudaSuccess || plan.s2_max <= 1) return err;
+    return launch_reduce_y(b.partials, b.splits + 1, R, H, b.y, st);
 }
 
 }  // namespace moe

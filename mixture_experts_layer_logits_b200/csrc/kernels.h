@@ -84,17 +84,16 @@ struct FfnBuffers {
     int32_t* splits;   // [2]: split counts the w13 and w2 kernels used
     int32_t* err;
 };
-// w13 (+ SwiGLU finalize when split) and w2.  between_gemms: if not null, recorded
-// on `st` after the w13 stage.  When the w2 split is > 1, y is left as partials:
-// the caller runs launch_combine (which reads them) or launch_reduce_y.
+// w13 (+ SwiGLU finalize when split) and w2 (+ y reduction when split): y is
+// complete when the launches finish.  between_gemms: if not null, recorded on
+// `st` after the w13 stage.
 cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, int I,
                                const FfnPlan& plan, cudaStream_t st,
                                cudaEvent_t between_gemms = nullptr);
 
-// out[t] = sum_j w[t,j] * y[t*k+j]; y is taken from w2's partials (summed in slice
-// order, rounded to bf16) when *splits > 1, else from the bf16 y.  splits may be null.
-cudaError_t launch_combine(const void* y, const float* partials, const int32_t* splits,
-                           const float* weights, int T, int k, int H, void* out, cudaStream_t st);
+// out[t] = sum_j w[t,j] * y[t*k+j] (k <= 16).
+cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
+                           cudaStream_t st);
 
 // act[p, f] = bf16(silu(sum_s gate_s) * sum_s up_s) when *splits > 1 (else no-op).
 cudaError_t launch_swiglu_finalize(const float* partials, const int32_t* splits, int R, int I,

@@ -244,10 +244,7 @@ moe_status_t moe_grouped_ffn(const moe_bf16_t* x, const moe_bf16_t* w13, const m
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     moe_status_t r = cuda_status(launch_build_tiles(expert_offsets, s.E, make_aux(ws, L, s), st));
     if (r != MOE_OK) return r;
-    r = run_ffn(x, w13, w2, permuted_rows, s, y, ws, L, st);
-    if (r != MOE_OK || L.plan.s2_max <= 1) return r;
-    return cuda_status(launch_reduce_y(at<float>(ws, L.partials), at<int32_t>(ws, L.splits),
-                                       s.T * s.top_k, s.H, y, st));
+    return run_ffn(x, w13, w2, permuted_rows, s, y, ws, L, st);
 }
 
 moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_shape_t s,
@@ -256,7 +253,7 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
     if (!y || !topk_weights || !out) return MOE_ERR_INVALID_ARG;
     if (!combine_shape_ok(s)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(y) || !aligned16(topk_weights) || !aligned16(out)) return MOE_ERR_MISALIGNED;
-    return cuda_status(launch_combine(y, nullptr, nullptr, topk_weights, s.T, s.top_k, s.H, out,
+    return cuda_status(launch_combine(y, topk_weights, s.T, s.top_k, s.H, out,
                                       static_cast<cudaStream_t>(stream)));
 }
 
@@ -293,9 +290,7 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
     if (r == MOE_OK) r = run_ffn(x, w13, w2, rows, s, y, ws, L, st, events ? events + 2 : nullptr);
     if (r == MOE_OK) r = mark(3);
     if (r == MOE_OK)
-        r = cuda_status(launch_combine(y, at<float>(ws, L.partials),
-                                       L.plan.s2_max > 1 ? at<int32_t>(ws, L.splits) + 1 : nullptr,
-                                       wts, s.T, s.top_k, s.H, out, st));
+        r = cuda_status(launch_combine(y, wts, s.T, s.top_k, s.H, out, st));
     if (r == MOE_OK) r = mark(4);
     return r;
 }
@@ -327,8 +322,9 @@ int moe_forward_kernel_count(moe_shape_t s)
     if (!ffn_shape_ok(s)) return 0;
     const long R = (long)s.T * s.top_k;
     const Layout L = layout_for(s);
-    // route(+permute) kernels, w13, [SwiGLU finalize], w2, combine
-    return (R <= kSmallRows ? 1 : 4) + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
+    // route(+permute) kernels, w13, [SwiGLU finalize], w2, [y reduction], combine
+    return (R <= kSmallRows ? 1 : 4) + 2 + (L.plan.s13_max > 1 ? 1 : 0) +
+           (L.plan.s2_max > 1 ? 1 : 0) + 1;
 }
 
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream)
