@@ -403,7 +403,7 @@ def routing_bench(args, w, rank, world, local, dev, pg):
                "kind": "oracle", "sample": f"all {T} tokens (route + permute) x {n} in {dt:.1f} s"}
     if rank == 0:
         all_bytes = route_bytes + perm_bytes
-        launches = 1 + (1 if R <= 4096 else 3)
+        launches = 1 + (1 if R <= 4096 else 2)
         line = {
             "metric": metric_name(w), "value": round(weak_scaling_value(world, T, ms), 2),
             "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,

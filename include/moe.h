@@ -140,7 +140,7 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
  * computes (same kernels, same bit-exact result).
  *
  * Scratch: a file-scope device array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES
- * (about 1 MiB) inside the library; every GPU on which the library is used holds
+ * (about 2 MiB) inside the library; every GPU on which the library is used holds
  * it until the process exits.  The caller still passes topk_ids, expert_offsets
  * and permuted_rows (device pointers, 16-byte aligned).
  * Limits: T*k <= MOE_PERMUTE_NOALLOC_MAX_ROWS and the moe_permute shape rules,
@@ -152,7 +152,7 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
  * streams or host threads, same device) race and may return wrong results;
  * order them on one stream. */
 #define MOE_PERMUTE_NOALLOC_MAX_ROWS (1 << 20)
-#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (1048576 + 32768 + 256)
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (2097152 + 32768 + 256)
 moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
                                  int32_t* expert_offsets, int32_t* permuted_rows,
                                  moe_stream_t stream);

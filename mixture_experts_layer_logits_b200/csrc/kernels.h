@@ -51,9 +51,9 @@ cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k,
                                        float* weights, int32_t* offsets, int32_t* rows,
                                        const PermuteAux& aux, cudaStream_t st);
 
-// Multi-CTA path: per-chunk counts, a scan over (expert, chunk), a per-chunk
-// stable scatter, tile list.
-constexpr int kChunkRows = 4096;
+// Multi-CTA path: per-chunk counts, then a per-chunk stable scatter whose CTAs
+// each scan the count table themselves (CTA 0 also writes offsets and tiles).
+constexpr int kChunkRows = 2048;
 cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                                  int32_t* rows, const PermuteAux& aux, cudaStream_t st);
 size_t large_permute_smem(int E);

@@ -323,7 +323,7 @@ int moe_forward_kernel_count(moe_shape_t s)
     const long R = (long)s.T * s.top_k;
     const Layout L = layout_for(s);
     // route(+permute) kernels, w13, [SwiGLU finalize], w2, [y reduction], combine
-    return (R <= kSmallRows ? 1 : 4) + 2 + (L.plan.s13_max > 1 ? 1 : 0) +
+    return (R <= kSmallRows ? 1 : 3) + 2 + (L.plan.s13_max > 1 ? 1 : 0) +
            (L.plan.s2_max > 1 ? 1 : 0) + 1;
 }
 

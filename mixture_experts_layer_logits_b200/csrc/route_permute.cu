@@ -3,17 +3,17 @@
 //
 // Routing ("softmax_sum", FlashInfer PR #3751 page "Optimizing TRTLLM-Gen MoE
 // routing", sections "1. dynamic thread-block size" and "performance numbers"):
-// one warp owns one token; each lane keeps E/32 logits in registers, the k
-// winners are taken one by one with a warp arg-max over (logit desc, expert asc)
-// keys, and the k weights are a softmax over the selected logits, summed in
-// selection order.  The pages size the routing CTA by token count to keep
+// one warp owns one token; each lane keeps E/32 logits in registers; a warp
+// bitonic sort of the lane maxima gives a threshold that leaves only a handful of
+// candidates, which are sorted by (logit desc, expert asc) keys; the k weights
+// are a softmax over the selected logits, summed in selection order.  The pages size the routing CTA by token count to keep
 // register pressure down; here the register footprint is fixed by the
 // per-lane value count V (a template), and the grid scales with T.
 //
 // Permutation: count -> exclusive scan -> stable scatter.  Ranks inside a warp
 // come from __match_any_sync peer masks, ranks across warps from a per-warp
 // count table and a column scan, ranks across CTAs from a per-chunk count table
-// scanned by one CTA, so the result (ascending expanded id inside every expert)
+// that every scatter CTA reads whole, so the result (ascending expanded id inside every expert)
 // never depends on atomic ordering.  No kernel waits on another CTA.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -35,68 +35,177 @@ __device__ __forceinline__ bool key_before(float va, int ia, float vb, int ib)
     return va > vb || (va == vb && ia < ib);
 }
 
+// Sorts one (value, index) key per lane across the warp so that lane 0 holds the
+// key that ranks first (larger value, then lower index).  Bitonic network with
+// the "ranks before" relation as the order; keys must be distinct (they are:
+// indices are unique).
+__device__ __forceinline__ void warp_sort_keys(float& v, int& i, int lane)
+{
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const float ov = __shfl_xor_sync(kFull, v, stride);
+            const int oi = __shfl_xor_sync(kFull, i, stride);
+            const bool take_first = ((lane & stride) == 0) == ((lane & size) == 0);
+            if (take_first == key_before(ov, oi, v, i)) {
+                v = ov;
+                i = oi;
+            }
+        }
+    }
+}
+
+// Sorts one float per lane across the warp, largest in lane 0.
+__device__ __forceinline__ float warp_sort_desc(float v, int lane)
+{
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const float o = __shfl_xor_sync(kFull, v, stride);
+            const bool take_max = ((lane & stride) == 0) == ((lane & size) == 0);
+            v = take_max ? fmaxf(v, o) : fminf(v, o);
+        }
+    }
+    return v;
+}
+
+// Expert held in value slot `s` of lane `lane`.  With VEC (E % 4 == 0, V % 4 == 0)
+// lane l loads float4 groups: slot 4m + c holds expert 128m + 4l + c; otherwise
+// slot s holds expert 32s + l.  Either way a lane's slots are in ascending expert
+// order.
+template <int V, bool VEC>
+__device__ __forceinline__ int slot_expert(int s, int lane)
+{
+    return VEC ? (s >> 2) * 128 + lane * 4 + (s & 3) : s * 32 + lane;
+}
+
 // Routes one token with the calling warp.  row: E logits.  Writes ids/weights
 // (k each) to global memory and, if ids_s != nullptr, the ids to shared memory.
-template <int V>
+// `cand` is this warp's shared scratch of 32 (value, index) pairs.
+//
+// Selection.  Let tau be the k-th largest of the 32 per-lane maxima: the k lanes
+// with the largest maxima hold k distinct experts with logit >= tau, so every
+// expert of the top k has logit >= tau.  The experts with logit >= tau are
+// gathered (one per lane) and sorted by (logit desc, expert asc); the first k
+// are the answer.  If more than 32 experts reach tau (ties, -inf rows), the
+// exact fallback takes the k winners one by one with a warp arg-max.
+template <int V, bool VEC>
 __device__ __forceinline__ void warp_route_token(const float* __restrict__ row, int E, int k,
                                                  int lane, int32_t* __restrict__ ids,
-                                                 float* __restrict__ weights, int* ids_s)
+                                                 float* __restrict__ weights, int* ids_s,
+                                                 float2* cand)
 {
     float v[V];
+    if (VEC) {
 #pragma unroll
-    for (int m = 0; m < V; ++m) {
-        const int e = m * 32 + lane;
-        v[m] = (e < E) ? __ldg(row + e) : -INFINITY;
-    }
-    uint32_t taken = 0;
-
-    // best not-yet-taken value of this lane; m ascending = expert ascending, so a
-    // strict '>' keeps the lower expert on equal values
-    auto lane_best = [&](float& bv, int& bi) {
-        bv = -INFINITY;
-        bi = kNoIndex;
+        for (int m = 0; m < V / 4; ++m) {
+            const int e = m * 128 + lane * 4;
+            float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            if (e < E) q = __ldg(reinterpret_cast<const float4*>(row + e));
+            v[4 * m] = q.x;
+            v[4 * m + 1] = q.y;
+            v[4 * m + 2] = q.z;
+            v[4 * m + 3] = q.w;
+        }
+    } else {
 #pragma unroll
         for (int m = 0; m < V; ++m) {
             const int e = m * 32 + lane;
-            const bool ok = e < E && !((taken >> m) & 1u);
-            if (ok && (bi == kNoIndex || v[m] > bv)) {
-                bv = v[m];
-                bi = e;
-            }
-        }
-    };
-
-    float bv;
-    int bi;
-    lane_best(bv, bi);
-    float my_l = 0.f;
-    int my_id = 0;
-    for (int j = 0; j < k; ++j) {
-        float wv = bv;
-        int wi = bi;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(kFull, wv, off);
-            const int oi = __shfl_xor_sync(kFull, wi, off);
-            if (key_before(ov, oi, wv, wi)) {
-                wv = ov;
-                wi = oi;
-            }
-        }
-        if (lane == j) {
-            my_l = wv;
-            my_id = wi;
-        }
-        if ((wi & 31) == lane) {  // the owner drops the winner and finds its next best
-            taken |= 1u << (wi >> 5);
-            lane_best(bv, bi);
+            v[m] = (e < E) ? __ldg(row + e) : -INFINITY;
         }
     }
-    // softmax over the selected logits; l_0 is the largest
+    // slots past E hold -inf; they are kept out of the candidates explicitly
+    float mv = -INFINITY;
+#pragma unroll
+    for (int m = 0; m < V; ++m) mv = fmaxf(mv, v[m]);
+    const float tau = __shfl_sync(kFull, warp_sort_desc(mv, lane), k - 1);
+
+    int c = 0;
+#pragma unroll
+    for (int m = 0; m < V; ++m) c += (slot_expert<V, VEC>(m, lane) < E && v[m] >= tau) ? 1 : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += n;
+    }
+    const int total = __shfl_sync(kFull, incl, 31);
+
+    float my_l = 0.f;
+    int my_id = 0;
+    if (total <= 32) {
+        int pos = incl - c;
+#pragma unroll
+        for (int m = 0; m < V; ++m) {
+            const int e = slot_expert<V, VEC>(m, lane);
+            if (e < E && v[m] >= tau) cand[pos++] = make_float2(v[m], __int_as_float(e));
+        }
+        __syncwarp();
+        float cv = -INFINITY;
+        int ci = kNoIndex - lane;  // distinct sentinels rank after every expert
+        if (lane < total) {
+            const float2 cc = cand[lane];
+            cv = cc.x;
+            ci = __float_as_int(cc.y);
+        }
+        __syncwarp();  // cand may be rewritten by this warp's next token
+        warp_sort_keys(cv, ci, lane);
+        my_l = cv;
+        my_id = ci;
+    } else {
+        uint32_t taken = 0;
+        // best not-yet-taken value of this lane; slots ascend with the expert, so a
+        // strict '>' keeps the lower expert on equal values
+        auto lane_best = [&](float& bv, int& bi) {
+            bv = -INFINITY;
+            bi = kNoIndex;
+#pragma unroll
+            for (int m = 0; m < V; ++m) {
+                const int e = slot_expert<V, VEC>(m, lane);
+                const bool ok = e < E && !((taken >> m) & 1u);
+                if (ok && (bi == kNoIndex || v[m] > bv)) {
+                    bv = v[m];
+                    bi = e;
+                }
+            }
+        };
+        float bv;
+        int bi;
+        lane_best(bv, bi);
+        for (int j = 0; j < k; ++j) {
+            float wv = bv;
+            int wi = bi;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, wv, off);
+                const int oi = __shfl_xor_sync(kFull, wi, off);
+                if (key_before(ov, oi, wv, wi)) {
+                    wv = ov;
+                    wi = oi;
+                }
+            }
+            if (lane == j) {
+                my_l = wv;
+                my_id = wi;
+            }
+            const int owner = VEC ? (wi & 127) >> 2 : (wi & 31);
+            if (owner == lane) {  // the owner drops the winner and finds its next best
+                const int slot = VEC ? (wi >> 7) * 4 + (wi & 3) : (wi >> 5);
+                taken |= 1u << slot;
+                lane_best(bv, bi);
+            }
+        }
+    }
+    // softmax over the selected logits; l_0 is the largest.  The sum is a fixed
+    // xor-tree over lanes 0..15 (lanes >= k contribute 0), so it is deterministic.
     const float l0 = __shfl_sync(kFull, my_l, 0);
     const float ex = (lane < k) ? expf(my_l - l0) : 0.f;
-    float sum = 0.f;
-    for (int j = 0; j < k; ++j) sum += __shfl_sync(kFull, ex, j);  // fixed order j = 0..k-1
+    float sum = ex;
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    sum = __shfl_sync(kFull, sum, 0);
     if (lane < k) {
         ids[lane] = my_id;
         weights[lane] = ex / sum;
@@ -210,21 +319,22 @@ __device__ __forceinline__ void warp_scatter(const int* ids_s, int r0, int r1, i
 
 // ----------------------------------------------------------------- kernels
 
-template <int V>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E,
-                                                    int k, int32_t* __restrict__ ids,
-                                                    float* __restrict__ weights)
+template <int V, bool VEC>
+__global__ void __launch_bounds__(256, 4) route_kernel(const float* __restrict__ logits, int T,
+                                                       int E, int k, int32_t* __restrict__ ids,
+                                                       float* __restrict__ weights)
 {
+    __shared__ float2 cand[8][32];
     pdl_wait();
     pdl_launch_dependents();
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
-    warp_route_token<V>(logits + (size_t)t * E, E, k, threadIdx.x & 31, ids + (size_t)t * k,
-                        weights + (size_t)t * k, nullptr);
+    warp_route_token<V, VEC>(logits + (size_t)t * E, E, k, threadIdx.x & 31, ids + (size_t)t * k,
+                             weights + (size_t)t * k, nullptr, cand[threadIdx.x >> 5]);
 }
 
 // One CTA: (route) + count + scan + stable scatter + tile list, for T*k <= kSmallRows.
-template <int V>
+template <int V, bool VEC>
 __global__ void __launch_bounds__(1024, 1)
     small_route_permute_kernel(const float* __restrict__ logits, int T, int E, int k,
                                int32_t* __restrict__ ids, float* __restrict__ weights,
@@ -242,9 +352,10 @@ __global__ void __launch_bounds__(1024, 1)
     pdl_launch_dependents();
 
     if (logits) {
+        __shared__ float2 cand[32][32];
         for (int t = warp; t < T; t += 32)
-            warp_route_token<V>(logits + (size_t)t * E, E, k, lane, ids + (size_t)t * k,
-                                weights + (size_t)t * k, ids_s + t * k);
+            warp_route_token<V, VEC>(logits + (size_t)t * E, E, k, lane, ids + (size_t)t * k,
+                                     weights + (size_t)t * k, ids_s + t * k, cand[warp]);
     } else {
         for (int r = threadIdx.x; r < R; r += blockDim.x) ids_s[r] = ids[r];
     }
@@ -292,38 +403,19 @@ __global__ void __launch_bounds__(1024) chunk_count_kernel(const int32_t* __rest
     for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = hist[e];
 }
 
-// counts[c][e] -> absolute position of chunk c's first row of expert e.
-__global__ void __launch_bounds__(1024) chunk_scan_kernel(int32_t* __restrict__ counts,
-                                                          int n_chunks, int E, int32_t* offsets,
-                                                          PermuteAux aux)
-{
-    __shared__ int sums[32];
-    pdl_wait();
-    pdl_launch_dependents();
-    const bool owns = threadIdx.x < E;
-    const int e = threadIdx.x;
-    int cnt = 0;
-    if (owns)
-        for (int c = 0; c < n_chunks; ++c) {
-            const int v = counts[(size_t)c * E + e];
-            counts[(size_t)c * E + e] = cnt;
-            cnt += v;
-        }
-    int total;
-    const int off = block_exclusive_scan(owns ? cnt : 0, sums, total);
-    if (owns) {
-        offsets[e] = off;
-        for (int c = 0; c < n_chunks; ++c) counts[(size_t)c * E + e] += off;
-    }
-    if (threadIdx.x == 0) offsets[E] = total;
-    write_tiles_and_reset(owns, e, cnt, off, aux, sums);
-}
-
+// One CTA per chunk of kChunkRows expanded rows.  Every CTA reads the whole
+// per-chunk count table (kept in L2) to get, for each expert e, the rows of e in
+// all chunks (-> the exclusive scan over experts, expert_offsets) and in the
+// chunks before its own (-> where its own rows of e start); then it ranks its
+// rows stably with per-warp tables and scatters them.  CTA 0 also writes
+// expert_offsets and the tile list.
 __global__ void __launch_bounds__(1024, 1)
-    chunk_scatter_kernel(const int32_t* __restrict__ ids, int R, int E,
-                         const int32_t* __restrict__ base, int32_t* __restrict__ rows_out)
+    chunk_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, int n_chunks,
+                         const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ rows_out, PermuteAux aux)
 {
     extern __shared__ int smem[];
+    __shared__ int sums[32];
     int* ids_s = smem;                 // kChunkRows
     int* table = smem + kChunkRows;    // [32][E]
     const int warp = threadIdx.x >> 5;
@@ -332,13 +424,41 @@ __global__ void __launch_bounds__(1024, 1)
     const int c0 = blockIdx.x * kChunkRows, n = min(kChunkRows, R - c0);
     for (int i = threadIdx.x; i < n; i += blockDim.x) ids_s[i] = ids[c0 + i];
     for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) table[i] = 0;
-    __syncthreads();
+
+    // per expert: rows in all chunks and rows in the chunks before this one; the
+    // loads of a batch are all issued before they are used
+    const bool owns = threadIdx.x < E;
+    const int e = threadIdx.x;
+    int total_e = 0, before_e = 0;
+    if (owns) {
+        constexpr int kBatch = 16;
+        for (int cb = 0; cb < n_chunks; cb += kBatch) {
+            int vals[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                vals[i] = (cb + i < n_chunks) ? __ldcg(counts + (size_t)(cb + i) * E + e) : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                total_e += vals[i];
+                if (cb + i < (int)blockIdx.x) before_e += vals[i];
+            }
+        }
+    }
+    int total;
+    const int off = block_exclusive_scan(owns ? total_e : 0, sums, total);
+    if (blockIdx.x == 0) {
+        if (owns) offsets[e] = off;
+        if (threadIdx.x == 0) offsets[E] = total;
+        write_tiles_and_reset(owns, e, total_e, off, aux, sums);
+    }
+    __syncthreads();  // ids_s and the zeroed table are complete
+
     constexpr int per_warp = kChunkRows / 32;
     const int r0 = min(n, warp * per_warp), r1 = min(n, r0 + per_warp);
     warp_count(ids_s, r0, r1, table + warp * E);
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = base[(size_t)blockIdx.x * E + e];
+    if (owns) {
+        int run = off + before_e;
         for (int w = 0; w < 32; ++w) {
             const int v = table[w * E + e];
             table[w * E + e] = run;
@@ -386,46 +506,63 @@ int values_per_lane(int E)
 
 }  // namespace
 
+template <int V>
+static cudaError_t launch_route_v(bool vec, const float* logits, int T, int E, int k, int32_t* ids,
+                                  float* weights, cudaStream_t st)
+{
+    const dim3 grid((T + 7) / 8), block(256);
+    if (vec && V >= 4)
+        return launch(route_kernel<V, (V >= 4)>, grid, block, 0, st, logits, T, E, k, ids, weights);
+    return launch(route_kernel<V, false>, grid, block, 0, st, logits, T, E, k, ids, weights);
+}
+
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights,
                          cudaStream_t st)
 {
-    const dim3 grid((T + 7) / 8), block(256);
+    const bool vec = (E % 4) == 0;
     switch (values_per_lane(E)) {
-    case 1: return launch(route_kernel<1>, grid, block, 0, st, logits, T, E, k, ids, weights);
-    case 2: return launch(route_kernel<2>, grid, block, 0, st, logits, T, E, k, ids, weights);
-    case 4: return launch(route_kernel<4>, grid, block, 0, st, logits, T, E, k, ids, weights);
-    case 8: return launch(route_kernel<8>, grid, block, 0, st, logits, T, E, k, ids, weights);
-    case 16: return launch(route_kernel<16>, grid, block, 0, st, logits, T, E, k, ids, weights);
-    default: return launch(route_kernel<32>, grid, block, 0, st, logits, T, E, k, ids, weights);
+    case 1: return launch_route_v<1>(vec, logits, T, E, k, ids, weights, st);
+    case 2: return launch_route_v<2>(vec, logits, T, E, k, ids, weights, st);
+    case 4: return launch_route_v<4>(vec, logits, T, E, k, ids, weights, st);
+    case 8: return launch_route_v<8>(vec, logits, T, E, k, ids, weights, st);
+    case 16: return launch_route_v<16>(vec, logits, T, E, k, ids, weights, st);
+    default: return launch_route_v<32>(vec, logits, T, E, k, ids, weights, st);
     }
 }
 
-template <int V>
+template <int V, bool VEC>
 static cudaError_t launch_small_v(const float* logits, int T, int E, int k, int32_t* ids,
                                   float* weights, int32_t* offsets, int32_t* rows,
                                   const PermuteAux& aux, cudaStream_t st)
 {
     const int R = T * k;
     const size_t smem = sizeof(int) * (size_t)(((R + 3) & ~3) + 32 * E);
-    cudaError_t err = cudaFuncSetAttribute(small_route_permute_kernel<V>,
+    cudaError_t err = cudaFuncSetAttribute(small_route_permute_kernel<V, VEC>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    return launch(small_route_permute_kernel<V>, dim3(1), dim3(1024), smem, st, logits, T, E, k,
-                  ids, weights, offsets, rows, aux);
+    return launch(small_route_permute_kernel<V, VEC>, dim3(1), dim3(1024), smem, st, logits, T, E,
+                  k, ids, weights, offsets, rows, aux);
 }
 
 cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k, int32_t* ids,
                                        float* weights, int32_t* offsets, int32_t* rows,
                                        const PermuteAux& aux, cudaStream_t st)
 {
+    const bool vec = (E % 4) == 0;
+#define MOE_SMALL(V)                                                                              \
+    (vec && (V) >= 4 ? launch_small_v<V, ((V) >= 4)>(logits, T, E, k, ids, weights, offsets, rows, \
+                                                     aux, st)                                     \
+                     : launch_small_v<V, false>(logits, T, E, k, ids, weights, offsets, rows, aux, \
+                                                st))
     switch (logits ? values_per_lane(E) : 1) {
-    case 1: return launch_small_v<1>(logits, T, E, k, ids, weights, offsets, rows, aux, st);
-    case 2: return launch_small_v<2>(logits, T, E, k, ids, weights, offsets, rows, aux, st);
-    case 4: return launch_small_v<4>(logits, T, E, k, ids, weights, offsets, rows, aux, st);
-    case 8: return launch_small_v<8>(logits, T, E, k, ids, weights, offsets, rows, aux, st);
-    case 16: return launch_small_v<16>(logits, T, E, k, ids, weights, offsets, rows, aux, st);
-    default: return launch_small_v<32>(logits, T, E, k, ids, weights, offsets, rows, aux, st);
+    case 1: return MOE_SMALL(1);
+    case 2: return MOE_SMALL(2);
+    case 4: return MOE_SMALL(4);
+    case 8: return MOE_SMALL(8);
+    case 16: return MOE_SMALL(16);
+    default: return MOE_SMALL(32);
     }
+#undef MOE_SMALL
 }
 
 size_t large_permute_smem(int E) { return sizeof(int) * (size_t)(kChunkRows + 32 * E); }
@@ -438,15 +575,12 @@ cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_
     cudaError_t err = launch(chunk_count_kernel, dim3(n_chunks), dim3(1024), sizeof(int) * E, st,
                              ids, R, E, aux.chunk_counts);
     if (err != cudaSuccess) return err;
-    err = launch(chunk_scan_kernel, dim3(1), dim3(1024), 0, st, aux.chunk_counts, n_chunks, E,
-                 offsets, aux);
-    if (err != cudaSuccess) return err;
     const size_t smem = large_permute_smem(E);
     err = cudaFuncSetAttribute(chunk_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);
     if (err != cudaSuccess) return err;
-    return launch(chunk_scatter_kernel, dim3(n_chunks), dim3(1024), smem, st, ids, R, E,
-                  (const int32_t*)aux.chunk_counts, rows);
+    return launch(chunk_scatter_kernel, dim3(n_chunks), dim3(1024), smem, st, ids, R, E, n_chunks,
+                  (const int32_t*)aux.chunk_counts, offsets, rows, aux);
 }
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, const PermuteAux& aux,
