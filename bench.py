@@ -44,9 +44,17 @@ if ROOT not in sys.path:
 FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes per launch of the dominant kernel from an ncu capture, keyed by
-# (workload, kernel); None until a capture of the current kernel exists.
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of a kernel from an ncu capture, keyed by
+# (workload, kernel) -- profiles/grouped_gemm_decode.md and
+# profiles/grouped_gemm_prefill_shape.md (prefill: the 16-expert capture scaled by
+# 8 to the 128-expert layer of the same per-expert shape).  Entries are removed
+# when the kernel changes, until it is captured again.
+NCU_TRAFFIC = {
+    ("decode", "w13"): 344_273_920,
+    ("decode", "w2"): 174_049_536,
+    ("prefill", "w13"): 3_489_796_096,
+    ("prefill", "w2"): 2_177_132_544,
+}
 
 
 def parse_args(argv=None):
