@@ -38,8 +38,8 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const uint4* __restrict__ y, const float* __restrict__ w, int T, int k, int H8,
                    uint4* __restrict__ out)
 {
+    pdl_launch_dependents();  // dependents wait for this grid's completion themselves
     pdl_wait();
-    pdl_launch_dependents();
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long)T * H8) return;
     const int t = (int)(idx / H8), h8 = (int)(idx % H8);
@@ -80,8 +80,8 @@ __global__ void __launch_bounds__(256)
     swiglu_finalize_kernel(const float4* __restrict__ partials, const int32_t* __restrict__ splits,
                            int R, int I4, uint2* __restrict__ act)
 {
+    pdl_launch_dependents();  // dependents wait for this grid's completion themselves
     pdl_wait();
-    pdl_launch_dependents();
     const int S = *splits;
     if (S <= 1) return;  // the GEMM wrote act itself
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(256)
     reduce_y_kernel(const float4* __restrict__ partials, const int32_t* __restrict__ splits,
                     int R, int H4, uint2* __restrict__ y)
 {
+    pdl_launch_dependents();  // dependents wait for this grid's completion themselves
     pdl_wait();
-    pdl_launch_dependents();
     const int S = *splits;
     if (S <= 1) return;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;

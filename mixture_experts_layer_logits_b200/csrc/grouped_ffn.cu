@@ -173,6 +173,24 @@ __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
 }
 
 
+// Tile list entries are read through L2 (they may be read before this grid's
+// dependency wait; see the kernel).
+__device__ __forceinline__ Tile load_tile(const Tile* p)
+{
+    const int4 lo = __ldcg(reinterpret_cast<const int4*>(p));
+    const int4 hi = __ldcg(reinterpret_cast<const int4*>(p) + 1);
+    Tile t;
+    t.expert = lo.x;
+    t.row_start = lo.y;
+    t.rows = lo.z;
+    t.first = lo.w;
+    t.count = hi.x;
+    t.pad[0] = hi.y;
+    t.pad[1] = hi.z;
+    t.pad[2] = hi.w;
+    return t;
+}
+
 __device__ __forceinline__ void flag_error(const FfnArgs& a, Aux* aux)
 {
     atomicExch(a.err, kDeviceErrorMagic);
@@ -221,10 +239,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = aux->tmem_base;
 
-    pdl_wait();  // routing, permutation, tile list (and, MODE 1, act) are ready
+    // Programmatic dependent launch.  w13 reads the tile list that the kernel
+    // right before it wrote, so all of it waits here.  w2 only needs its
+    // predecessor (the SwiGLU finalize, or w13) for the act rows it loads and for
+    // the partials region its epilogue overwrites: its producer waits right before
+    // the first act load and its epilogue before its first store, so the weight
+    // loads of its first stages overlap the end of the w13 stage.  The tile list
+    // it reads before waiting was written two or more launches earlier: w2 is
+    // only launched once every w13 CTA has passed its own wait, i.e. after the
+    // permutation and everything before it completed.  It is read with L2 loads.
+    if (MODE == 0) pdl_wait();
     pdl_launch_dependents();
 
-    const int ntiles = *a.num_tiles;
+    const int ntiles = __ldcg(a.num_tiles);
     const int s_want = split_count(a, ntiles);
     const int kt_per_split = (a.num_kt + s_want - 1) / s_want;
     const int S = (a.num_kt + kt_per_split - 1) / kt_per_split;  // every slice non-empty
@@ -242,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto decode = [&](int u, int& split, int& tile, int& fb) {
         split = u % S;
         const int rest = u / S;
-        const Tile& probe = a.tiles[rest / a.fb_count];
+        const Tile probe = load_tile(a.tiles + rest / a.fb_count);
         const int local = rest - a.fb_count * probe.first;
         fb = local / probe.count;
         tile = probe.first + local % probe.count;
@@ -260,10 +287,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued[16];
             for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
             bool ok = true;
+            bool dep_ready = MODE == 0;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 int split, tile, fb;
                 decode(u, split, tile, fb);
-                const Tile t = a.tiles[tile];
+                const Tile t = load_tile(a.tiles + tile);
                 const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
                 for (int kt = kt0; kt < kt1; ++kt) {
                     if (!mbar_wait(&aux->empty[stage], phase ^ 1u, abort_flag)) {
@@ -287,6 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(st, &tm_w, &aux->full[stage], kt * kBK, row, pol);
                         tma_load_2d(st + kATileBytes, &tm_w, &aux->full[stage], kt * kBK,
                                     row + kBM, pol);
+                        if (!dep_ready) {  // act comes from the previous kernel
+                            pdl_wait();
+                            dep_ready = true;
+                        }
                         tma_load_2d_nohint(st + 2 * kATileBytes, &tm_act, &aux->full[stage],
                                            kt * kBK, t.row_start);
                     }
@@ -307,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            if (!dep_ready) pdl_wait();  // (no unit here) the grid still depends on it
             if (!ok || *abort_flag) {
                 // let every TMA load already issued land before the CTA can exit
                 for (int s = 0; s < C::kStages; ++s)
@@ -327,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++lu) {
                 int split, tile, fb;
                 decode(u, split, tile, fb);
-                const Tile t = a.tiles[tile];
+                const Tile t = load_tile(a.tiles + tile);
                 const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
                 const int b = lu % C::kNBuf;
                 const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
@@ -388,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int q_unit0 = q;
                 q += kt1 - kt0;
                 if (kt >= kt1) continue;
-                const Tile t = a.tiles[tile];
+                const Tile t = load_tile(a.tiles + tile);
                 if (tile != cur_tile) {
                     __syncwarp();  // earlier copies' addresses are all issued
                     for (int j = lane; j < t.rows; j += 32)
@@ -428,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         if (warp < kEpiWarp0) goto teardown;
+        if (MODE == 1) pdl_wait();  // the outputs and partials the predecessor reads
         const int grp = (warp - kEpiWarp0) >> 2;  // token-column half
         const int q = warp & 3;                 // TMEM lane quarter
         const int f_local = q * 32 + lane;      // feature inside the 128-row block
@@ -438,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++lu) {
             int split, tile, fb;
             decode(u, split, tile, fb);
-            const Tile t = a.tiles[tile];
+            const Tile t = load_tile(a.tiles + tile);
             const int b = lu % C::kNBuf;
             const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
             const bool got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
