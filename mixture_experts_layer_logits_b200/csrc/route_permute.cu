@@ -92,12 +92,9 @@ __device__ __forceinline__ int slot_expert(int s, int lane)
 // are the answer.  If more than 32 experts reach tau (ties, -inf rows), the
 // exact fallback takes the k winners one by one with a warp arg-max.
 template <int V, bool VEC>
-__device__ __forceinline__ void warp_route_token(const float* __restrict__ row, int E, int k,
-                                                 int lane, int32_t* __restrict__ ids,
-                                                 float* __restrict__ weights, int* ids_s,
-                                                 float2* cand)
+__device__ __forceinline__ void warp_load_row(const float* __restrict__ row, int E, int lane,
+                                              float (&v)[V])
 {
-    float v[V];
     if (VEC) {
 #pragma unroll
         for (int m = 0; m < V / 4; ++m) {
@@ -116,6 +113,14 @@ __device__ __forceinline__ void warp_route_token(const float* __restrict__ row, 
             v[m] = (e < E) ? __ldg(row + e) : -INFINITY;
         }
     }
+}
+
+template <int V, bool VEC>
+__device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, int k, int lane,
+                                                  int32_t* __restrict__ ids,
+                                                  float* __restrict__ weights, int* ids_s,
+                                                  float2* cand)
+{
     // slots past E hold -inf; they are kept out of the candidates explicitly
     float mv = -INFINITY;
 #pragma unroll
@@ -211,6 +216,17 @@ __device__ __forceinline__ void warp_route_token(const float* __restrict__ row, 
         weights[lane] = ex / sum;
         if (ids_s) ids_s[lane] = my_id;
     }
+}
+
+template <int V, bool VEC>
+__device__ __forceinline__ void warp_route_token(const float* __restrict__ row, int E, int k,
+                                                 int lane, int32_t* __restrict__ ids,
+                                                 float* __restrict__ weights, int* ids_s,
+                                                 float2* cand)
+{
+    float v[V];
+    warp_load_row<V, VEC>(row, E, lane, v);
+    warp_select_token<V, VEC>(v, E, k, lane, ids, weights, ids_s, cand);
 }
 
 // Exclusive scan of one int per thread over the whole CTA (blockDim.x a
@@ -353,25 +369,35 @@ __global__ void __launch_bounds__(1024, 1)
 
     if (logits) {
         __shared__ float2 cand[32][32];
-        for (int t = warp; t < T; t += 32)
-            warp_route_token<V, VEC>(logits + (size_t)t * E, E, k, lane, ids + (size_t)t * k,
-                                     weights + (size_t)t * k, ids_s + t * k, cand[warp]);
+        // a warp's next token is loaded while its current one is selected
+        float v[V];
+        if (warp < T) warp_load_row<V, VEC>(logits + (size_t)warp * E, E, lane, v);
+        for (int t = warp; t < T; t += 32) {
+            float nv[V];
+            if (t + 32 < T) warp_load_row<V, VEC>(logits + (size_t)(t + 32) * E, E, lane, nv);
+            warp_select_token<V, VEC>(v, E, k, lane, ids + (size_t)t * k, weights + (size_t)t * k,
+                                      ids_s + t * k, cand[warp]);
+#pragma unroll
+            for (int m = 0; m < V; ++m) v[m] = nv[m];
+        }
     } else {
         for (int r = threadIdx.x; r < R; r += blockDim.x) ids_s[r] = ids[r];
     }
-    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) table[i] = 0;
+    // counting warps: as many as there are 32-row groups, up to 32
+    const int W = min(32, (R + 31) / 32);
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) table[i] = 0;
     __syncthreads();
 
-    const int per_warp = (R + 31) / 32;
-    const int r0 = min(R, warp * per_warp), r1 = min(R, r0 + per_warp);
-    warp_count(ids_s, r0, r1, table + warp * E);
+    const int per_warp = (R + W - 1) / W;
+    const int r0 = min(R, warp * per_warp), r1 = warp < W ? min(R, r0 + per_warp) : r0;
+    if (warp < W) warp_count(ids_s, r0, r1, table + warp * E);
     __syncthreads();
 
     const bool owns = threadIdx.x < E;
     const int e = threadIdx.x;
     int cnt = 0;
     if (owns)
-        for (int w = 0; w < 32; ++w) {
+        for (int w = 0; w < W; ++w) {
             const int c = table[w * E + e];
             table[w * E + e] = cnt;
             cnt += c;
@@ -380,13 +406,13 @@ __global__ void __launch_bounds__(1024, 1)
     const int off = block_exclusive_scan(owns ? cnt : 0, sums, total);
     if (owns) {
         offsets[e] = off;
-        for (int w = 0; w < 32; ++w) table[w * E + e] += off;
+        for (int w = 0; w < W; ++w) table[w * E + e] += off;
     }
     if (threadIdx.x == 0) offsets[E] = total;
     write_tiles_and_reset(owns, e, cnt, off, aux, sums);
     __syncthreads();
 
-    warp_scatter(ids_s, r0, r1, 0, table + warp * E, rows_out);
+    if (warp < W) warp_scatter(ids_s, r0, r1, 0, table + warp * E, rows_out);
 }
 
 __global__ void __launch_bounds__(1024) chunk_count_kernel(const int32_t* __restrict__ ids, int R,
