@@ -678,19 +678,6 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
                                const FfnPlan& plan, cudaStream_t st, cudaEvent_t between_gemms)
 {
     const int R = T * k;
-    if (plan.nt == 256 && plan.s13_max == 1 && plan.s2_max == 1) {
-        // tensor-bound shapes: CTA pairs, when the device can co-schedule them
-        const int pairs = min(plan.grid / 2, pair_kernel_max_pairs(plan.grid));
-        if (pairs > 0) {
-            CUtensorMap th, tw, ta;
-            cudaError_t err = make_tmap(&th, b.w13, (uint64_t)E * 2 * I, (uint64_t)H, 64);
-            if (err == cudaSuccess) err = make_tmap(&tw, b.w2, (uint64_t)E * H, (uint64_t)I, kBM);
-            if (err == cudaSuccess)
-                err = make_tmap(&ta, b.act, (uint64_t)R, (uint64_t)I, 128);
-            if (err != cudaSuccess) return err;
-            return launch_grouped_ffn_pair(b, th, tw, ta, T, k, H, I, pairs, st, between_gemms);
-        }
-    }
     CUtensorMap tw13, tw2, tact;
     cudaError_t err = make_tmap(&tw13, b.w13, (uint64_t)E * 2 * I, (uint64_t)H, kBM);
     if (err == cudaSuccess) err = make_tmap(&tw2, b.w2, (uint64_t)E * H, (uint64_t)I, kBM);

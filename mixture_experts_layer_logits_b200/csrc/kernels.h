@@ -91,15 +91,6 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
                                const FfnPlan& plan, cudaStream_t st,
                                cudaEvent_t between_gemms = nullptr);
 
-// Large-batch grouped FFN on CTA pairs (cta_group::2): 256-token tiles, no split.
-// tw13_half: w13 as [E*2I, H] with a 64-row box; tw2: w2 as [E*H, I] with a 128-row
-// box; tact: act as [R, I] with a 128-row box.
-int pair_kernel_max_pairs(int num_sms);
-cudaError_t launch_grouped_ffn_pair(const FfnBuffers& b, const CUtensorMap& tw13_half,
-                                    const CUtensorMap& tw2, const CUtensorMap& tact, int T, int k,
-                                    int H, int I, int pairs, cudaStream_t st,
-                                    cudaEvent_t between_gemms);
-
 // out[t] = sum_j w[t,j] * y[t*k+j] (k <= 16).
 cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
                            cudaStream_t st);
