@@ -5,8 +5,9 @@
 //                    "FP32 partials" section of the FlashInfer PR #5586 page, applied
 //                    to the top-k combine).
 //   swiglu finalize  act[p, f] = bf16(silu(sum_s gate_s) * sum_s up_s) for a split w13.
-//   reduce y         y[r, h] = bf16(sum_s partial_s[r, h]) for a split w2 (before the
-//                    combine, or for moe_grouped_ffn's y).
+//   reduce y         y[r, h] = bf16(sum_s partial_s[r, h]) for a split w2 whose y is
+//                    wanted on its own (moe_grouped_ffn).
+//   combine from partials   the two above in one kernel, for moe_forward.
 //
 // Each thread moves 16-byte vectors and issues all of its loads before using any
 // (these kernels are short and latency-bound at decode sizes); the split count
@@ -73,6 +74,72 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < 4; ++i) q[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
     out[idx] = o;
+}
+
+// Combine straight from w2's split-K partials.  Block = one token t and 256
+// consecutive hidden elements, 64 threads per selected expert j: thread (j, c)
+// rebuilds 4 elements of y[t*k + j] as bf16(sum_s partial_s), every slice's load
+// in flight (or reads them from y when w2 ran unsplit); then, per element, the
+// k rows are accumulated in j order with the same fma chain as combine_kernel.
+// The result is bit-identical to reduce_y followed by combine_kernel.
+__global__ void __launch_bounds__(1024)
+    combine_partials_kernel(const float4* __restrict__ partials, const int32_t* __restrict__ splits,
+                            const uint2* __restrict__ y, const float* __restrict__ w, int T,
+                            int k, int H4, uint2* __restrict__ out)
+{
+    __shared__ float4 yrow[kMaxK][64];
+    __shared__ float wrow[kMaxK];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int S = *splits;
+    const int t = blockIdx.x;
+    const int c = threadIdx.x & 63, j = threadIdx.x >> 6;  // blockDim = 64 * k
+    const int h4 = blockIdx.y * 64 + c;
+    const long R = (long)T * k;
+    const long r = (long)t * k + j;
+    if (c == 0) wrow[j] = __ldg(w + r);
+    if (h4 < H4) {
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        if (S > 1) {
+            float4 pv[kMaxSplits];
+#pragma unroll
+            for (int s = 0; s < kMaxSplits; ++s)
+                if (s < S) pv[s] = __ldcs(partials + ((size_t)s * R + r) * H4 + h4);
+#pragma unroll
+            for (int s = 0; s < kMaxSplits; ++s) {  // slice order
+                if (s < S) {
+                    a[0] += pv[s].x; a[1] += pv[s].y; a[2] += pv[s].z; a[3] += pv[s].w;
+                }
+            }
+            a[0] = __bfloat162float(__float2bfloat16_rn(a[0]));
+            a[1] = __bfloat162float(__float2bfloat16_rn(a[1]));
+            a[2] = __bfloat162float(__float2bfloat16_rn(a[2]));
+            a[3] = __bfloat162float(__float2bfloat16_rn(a[3]));
+        } else {
+            const uint2 v = __ldcs(y + r * H4 + h4);
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+            const float2 f0 = __bfloat1622float2(p[0]), f1 = __bfloat1622float2(p[1]);
+            a[0] = f0.x; a[1] = f0.y; a[2] = f1.x; a[3] = f1.y;
+        }
+        yrow[j][c] = make_float4(a[0], a[1], a[2], a[3]);
+    }
+    __syncthreads();
+    if (j == 0 && h4 < H4) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int jj = 0; jj < k; ++jj) {  // j ascending: the fixed summation order
+            const float4 v = yrow[jj][c];
+            const float wj = wrow[jj];
+            acc[0] = fmaf(wj, v.x, acc[0]);
+            acc[1] = fmaf(wj, v.y, acc[1]);
+            acc[2] = fmaf(wj, v.z, acc[2]);
+            acc[3] = fmaf(wj, v.w, acc[3]);
+        }
+        uint2 o;
+        __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);
+        q[0] = __floats2bfloat162_rn(acc[0], acc[1]);
+        q[1] = __floats2bfloat162_rn(acc[2], acc[3]);
+        out[(size_t)t * H4 + h4] = o;
+    }
 }
 
 // partials: [S, R, 2I] fp32 (gate columns [0, I), up columns [I, 2I)); 4 features per thread
@@ -164,6 +231,26 @@ cudaError_t launch_combine(const void* y, const float* weights, int T, int k, in
     const int H8 = H / 8;
     return launch_1d(combine_kernel, (long)T * H8, st, static_cast<const uint4*>(y), weights, T, k,
                      H8, static_cast<uint4*>(out));
+}
+
+cudaError_t launch_combine_partials(const float* partials, const int32_t* splits, const void* y,
+                                   const float* weights, int T, int k, int H, void* out,
+                                   cudaStream_t st)
+{
+    if (T == 0) return cudaSuccess;
+    const int H4 = H / 4;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)T, (unsigned)((H4 + 63) / 64));
+    cfg.blockDim = dim3((unsigned)(64 * k));
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_partials_kernel, reinterpret_cast<const float4*>(partials),
+                              splits, static_cast<const uint2*>(y), weights, T, k, H4,
+                              static_cast<uint2*>(out));
 }
 
 cudaError_t launch_swiglu_finalize(const float* partials, const int32_t* splits, int R, int I,

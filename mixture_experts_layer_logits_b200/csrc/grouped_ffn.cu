@@ -675,7 +675,8 @@ FfnPlan plan_ffn(int T, int E, int k, int H, int I, int num_sms)
 }
 
 cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, int I,
-                               const FfnPlan& plan, cudaStream_t st, cudaEvent_t between_gemms)
+                               const FfnPlan& plan, cudaStream_t st, cudaEvent_t between_gemms,
+                               bool reduce_y)
 {
     const int R = T * k;
     CUtensorMap tw13, tw2, tact;
@@ -723,7 +724,7 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
     a.fb_count = (H / kBM + 1) / 2;
     a.s_max = plan.s2_max;
     err = launch_nt<1>(plan.nt, tw2, tact, a, plan.grid, st);
-    if (err != cudaSuccess || plan.s2_max <= 1) return err;
+    if (err != cudaSuccess || plan.s2_max <= 1 || !reduce_y) return err;
     return launch_reduce_y(b.partials, b.splits + 1, R, H, b.y, st);
 }
 

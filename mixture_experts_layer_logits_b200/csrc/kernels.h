@@ -84,16 +84,24 @@ struct FfnBuffers {
     int32_t* splits;   // [2]: split counts the w13 and w2 kernels used
     int32_t* err;
 };
-// w13 (+ SwiGLU finalize when split) and w2 (+ y reduction when split): y is
-// complete when the launches finish.  between_gemms: if not null, recorded on
-// `st` after the w13 stage.
+// w13 (+ SwiGLU finalize when split) and w2 (+ y reduction when split and
+// reduce_y): y is complete when the launches finish, unless reduce_y is false,
+// in which case a split w2 leaves its partials for launch_combine_partials.
+// between_gemms: if not null, recorded on `st` after the w13 stage.
 cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, int I,
                                const FfnPlan& plan, cudaStream_t st,
-                               cudaEvent_t between_gemms = nullptr);
+                               cudaEvent_t between_gemms = nullptr, bool reduce_y = true);
 
 // out[t] = sum_j w[t,j] * y[t*k+j] (k <= 16).
 cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
                            cudaStream_t st);
+
+// The combine reading w2's split-K partials (k <= 16, splits <= 8): y[r] =
+// bf16(sum_s partial_s[r]) in slice order (y itself when *splits <= 1), then
+// the combine.  Used when w2 may be split.
+cudaError_t launch_combine_partials(const float* partials, const int32_t* splits, const void* y,
+                                   const float* weights, int T, int k, int H, void* out,
+                                   cudaStream_t st);
 
 // act[p, f] = bf16(silu(sum_s gate_s) * sum_s up_s) when *splits > 1 (else no-op).
 cudaError_t launch_swiglu_finalize(const float* partials, const int32_t* splits, int R, int I,

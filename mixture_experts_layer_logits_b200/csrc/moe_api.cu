@@ -166,7 +166,7 @@ moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, cons
 
 moe_status_t run_ffn(const void* x, const void* w13, const void* w2, const int32_t* rows,
                      const moe_shape_t& s, void* y, void* ws, const Layout& L, cudaStream_t st,
-                     void* const* mid_event = nullptr)
+                     void* const* mid_event = nullptr, bool reduce_y = true)
 {
     FfnBuffers b;
     b.x = x;
@@ -184,7 +184,7 @@ moe_status_t run_ffn(const void* x, const void* w13, const void* w2, const int32
     plan.grid = device_sms();
     return cuda_status(launch_grouped_ffn(
         b, s.T, s.E, s.top_k, s.H, s.I, plan, st,
-        mid_event ? static_cast<cudaEvent_t>(mid_event[0]) : nullptr));
+        mid_event ? static_cast<cudaEvent_t>(mid_event[0]) : nullptr, reduce_y));
 }
 
 }  // namespace
@@ -287,10 +287,16 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
     moe_status_t r = mark(0);
     if (r == MOE_OK) r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st);
     if (r == MOE_OK) r = mark(1);
-    if (r == MOE_OK) r = run_ffn(x, w13, w2, rows, s, y, ws, L, st, events ? events + 2 : nullptr);
+    // a split w2 is reduced inside the combine (one launch fewer)
+    const bool split2 = L.plan.s2_max > 1;
+    if (r == MOE_OK)
+        r = run_ffn(x, w13, w2, rows, s, y, ws, L, st, events ? events + 2 : nullptr, !split2);
     if (r == MOE_OK) r = mark(3);
     if (r == MOE_OK)
-        r = cuda_status(launch_combine(y, wts, s.T, s.top_k, s.H, out, st));
+        r = cuda_status(split2 ? launch_combine_partials(at<float>(ws, L.partials),
+                                                         at<int32_t>(ws, L.splits) + 1, y, wts, s.T,
+                                                         s.top_k, s.H, out, st)
+                               : launch_combine(y, wts, s.T, s.top_k, s.H, out, st));
     if (r == MOE_OK) r = mark(4);
     return r;
 }
@@ -322,9 +328,8 @@ int moe_forward_kernel_count(moe_shape_t s)
     if (!ffn_shape_ok(s)) return 0;
     const long R = (long)s.T * s.top_k;
     const Layout L = layout_for(s);
-    // route(+permute) kernels, w13, [SwiGLU finalize], w2, [y reduction], combine
-    return (R <= kSmallRows ? 1 : 3) + 2 + (L.plan.s13_max > 1 ? 1 : 0) +
-           (L.plan.s2_max > 1 ? 1 : 0) + 1;
+    // route(+permute) kernels, w13, [SwiGLU finalize], w2, combine
+    return (R <= kSmallRows ? 1 : 3) + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
 }
 
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream)
