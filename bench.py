@@ -45,16 +45,9 @@ FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of a kernel from an ncu capture, keyed by
-# (workload, kernel) -- profiles/grouped_gemm_decode.md and
-# profiles/grouped_gemm_prefill_shape.md (prefill: the 16-expert capture scaled by
-# 8 to the 128-expert layer of the same per-expert shape).  Entries are removed
-# when the kernel changes, until it is captured again.
-NCU_TRAFFIC = {
-    ("decode", "w13"): 344_273_920,
-    ("decode", "w2"): 174_049_536,
-    ("prefill", "w13"): 3_489_796_096,
-    ("prefill", "w2"): 2_177_132_544,
-}
+# (workload, kernel), from the summaries under profiles/.  An entry is removed
+# when its kernel changes, until it is captured again.
+NCU_TRAFFIC = {}
 
 
 def parse_args(argv=None):
@@ -132,6 +125,11 @@ def stage_work(w, n_touched):
                     flops=2 * R * 2 * I * H),
         "w2": dict(bytes=n_touched * H * I * 2 + R * I * 2 + R * H * 2, flops=2 * R * H * I),
         "combine": dict(bytes=R * H * 2 + R * 4 + T * H * 2, flops=0),
+        # w13 + w2 + combine as one launch: act and y never need to reach HBM, so
+        # the algorithmic bytes are the touched weights, x, the routing weights and
+        # permuted rows, and out
+        "fused_ffn": dict(bytes=n_touched * 3 * I * H * 2 + T * H * 2 + R * 8 + T * H * 2,
+                          flops=2 * R * 2 * I * H + 2 * R * H * I),
     }
 
 
@@ -545,9 +543,13 @@ def main(argv=None):
         moe.moe_forward_timed(x, logits, w13, w2, k, sev[i], ws=ws, out=out, topk_ids=ids,
                               topk_weights=wts, expert_offsets=off, permuted_rows=rows)
     barrier()
-    names = ["route_permute", "w13", "w2", "combine"]
-    stage_ms = {n: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(KB))
-                for j, n in enumerate(names)}
+    fused = moe.moe_forward_fused(T, E, k, H, I)
+    if fused:  # events 2..4 all follow the one FFN + combine launch
+        spans = {"route_permute": (0, 1), "fused_ffn": (1, 4)}
+    else:
+        spans = {"route_permute": (0, 1), "w13": (1, 2), "w2": (2, 3), "combine": (3, 4)}
+    stage_ms = {n: statistics.mean(sev[i][a].elapsed_time(sev[i][b]) for i in range(KB))
+                for n, (a, b) in spans.items()}
     stage_ms = {n: slowest(v) for n, v in stage_ms.items()}
 
     # ---- pass C: end to end from pinned host memory
@@ -574,7 +576,7 @@ def main(argv=None):
     # ---- roofline of the dominant kernel
     peaks, peak_kind = load_peaks()
     work = stage_work(w, n_touched)
-    dominant = max(("w13", "w2", "route_permute", "combine"), key=lambda n: stage_ms[n])
+    dominant = max(stage_ms, key=lambda n: stage_ms[n])
     sustained = K * ms > 1000.0  # a seconds-long timed region runs at the power-capped clock
     roof = roofline_entry(dominant, work[dominant], stage_ms[dominant], peaks, peak_kind,
                           sustained, NCU_TRAFFIC.get((w.name, dominant)))

@@ -113,7 +113,13 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
 /* The whole layer: route -> permute -> ffn -> combine, one stream, no host sync.
  * x bf16 [T, H], logits fp32 [T, E], w13 bf16 [E, 2I, H], w2 bf16 [E, H, I]
  * -> out bf16 [T, H].  topk_ids, topk_weights, expert_offsets and permuted_rows
- * are optional outputs: pass NULL to keep them inside the workspace. */
+ * are optional outputs: pass NULL to keep them inside the workspace.
+ * For weight-streaming shapes (T <= 64, see moe_forward_fused) w13, w2 and the
+ * combine run as ONE persistent launch whose CTAs hand act rows and finished y
+ * rows to each other through arrival counters in the workspace; its result is
+ * bit-identical to the multi-launch path, which MOE_DISABLE_FUSED=1 in the
+ * environment selects instead.  Either way every wait is bounded (2 s; then
+ * moe_device_status reports MOE_ERR_DEVICE_TIMEOUT). */
 moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
                          const moe_bf16_t* w2, moe_shape_t shape, moe_bf16_t* out,
                          int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
@@ -124,8 +130,10 @@ moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf1
  * events[i] (cudaEvent_t, created by the caller) on `stream` at the stage
  * boundaries: [0] before routing, [1] after route+permute, [2] after the
  * w13/SwiGLU kernel, [3] after the w2 kernel, [4] after the combine.  n_events
- * must be 5.  A recorded event is a stream operation, so the launch overlap
- * between the stages it separates is lost while measuring. */
+ * must be 5.  When the FFN and combine are one launch (moe_forward_fused),
+ * events [2], [3] and [4] are all recorded after it.  A recorded event is a
+ * stream operation, so the launch overlap between the stages it separates is
+ * lost while measuring. */
 moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
                                const moe_bf16_t* w2, moe_shape_t shape, moe_bf16_t* out,
                                int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
@@ -159,6 +167,10 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
 
 /* Number of kernels one moe_forward call launches for `shape` (0 if unsupported). */
 int moe_forward_kernel_count(moe_shape_t shape);
+
+/* 1 if moe_forward runs w13, w2 and the combine of `shape` as one persistent
+ * launch (T <= 64 and T*k <= 4096, unless MOE_DISABLE_FUSED=1), else 0. */
+int moe_forward_fused(moe_shape_t shape);
 
 /* Waits for `stream`, then reads and clears the device error word kept in the
  * workspace.  MOE_ERR_DEVICE_TIMEOUT means a kernel gave up on a bounded

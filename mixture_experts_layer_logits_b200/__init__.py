@@ -18,6 +18,7 @@ import torch
 __all__ = [
     "MoeError", "Shape", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_forward_timed", "moe_forward_kernel_count",
+    "moe_forward_fused",
     "moe_device_status", "library_path", "load_library",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ERR_MISALIGNED",
     "MOE_ERR_WORKSPACE_TOO_SMALL", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
@@ -74,6 +75,8 @@ def load_library():
                                       ctypes.c_size_t, _vp, ctypes.POINTER(_vp), ctypes.c_int]
     lib.moe_forward_kernel_count.argtypes = [Shape]
     lib.moe_forward_kernel_count.restype = ctypes.c_int
+    lib.moe_forward_fused.argtypes = [Shape]
+    lib.moe_forward_fused.restype = ctypes.c_int
     lib.moe_device_status.argtypes = [_vp, ctypes.c_size_t, _vp]
     for fn in (lib.moe_route, lib.moe_permute, lib.moe_grouped_ffn, lib.moe_combine,
                lib.moe_forward, lib.moe_forward_timed, lib.moe_device_status):
@@ -234,6 +237,11 @@ def moe_forward_timed(x, logits, w13, w2, top_k: int, events, ws=None, out=None,
 
 def moe_forward_kernel_count(T: int, E: int, top_k: int, H: int, I: int) -> int:
     return int(load_library().moe_forward_kernel_count(Shape(T, E, top_k, H, I)))
+
+
+def moe_forward_fused(T: int, E: int, top_k: int, H: int, I: int) -> bool:
+    """True if moe_forward runs the FFN and the combine as one persistent launch."""
+    return bool(load_library().moe_forward_fused(Shape(T, E, top_k, H, I)))
 
 
 def moe_device_status(ws: torch.Tensor) -> int:

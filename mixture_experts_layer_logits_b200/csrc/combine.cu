@@ -16,6 +16,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gemm_common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -23,12 +24,7 @@ namespace moe {
 
 namespace {
 
-// silu(g) * u with the same fast exponential and reciprocal as the GEMM epilogue
-// (the product is rounded to bf16).
-__device__ __forceinline__ float silu_mul(float g, float u)
-{
-    return g * __frcp_rn(1.0f + __expf(-g)) * u;
-}
+using gemm::silu_mul;  // the GEMM epilogue's SwiGLU, bit for bit
 
 constexpr int kMaxK = 16;
 constexpr int kMaxSplits = 8;

@@ -52,6 +52,7 @@
 
 #include <mutex>
 
+#include "gemm_common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -59,16 +60,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kBM = 128;        // weight rows per tile (MMA M)
-constexpr int kBK = 64;         // K elements per stage (one 128-byte swizzle row)
-constexpr int kUmmaK = 16;      // K per tcgen05.mma (bf16)
-constexpr int kThreads = 512;   // 16 warps, roles below
-constexpr int kGatherWarps = 6;  // warps 2..7
-constexpr int kEpiWarp0 = 8;     // warps 8..15: two epilogue groups of four
-constexpr int kPrefetch = 4;     // weight K-tiles brought to L2 ahead of their TMA
-constexpr int kStageRows = 8;    // token rows per epilogue staging buffer
-constexpr int kStageRowBytes = 512;  // one token row: 256 bf16 outputs
-constexpr int kATileBytes = kBM * kBK * 2;
+using namespace gemm;
 
 struct FfnArgs {
     const __nv_bfloat16* x;
@@ -87,109 +79,6 @@ struct FfnArgs {
     int min_kt_per_split;
     int weights_evict_first;  // weights are streamed once (few tokens per expert)
 };
-
-template <int MODE, int NT>
-struct Cfg {
-    static constexpr int kNA = 2;                                  // A tiles per stage
-    static constexpr int kBTileBytes = NT * kBK * 2;
-    static constexpr int kStageBytes = kNA * kATileBytes + kBTileBytes;
-    // shared memory: 1 KB alignment slack | ring | epilogue staging | Aux | token offsets
-    static constexpr int kMaxSmem = 232448;  // 227 KB per CTA
-    static constexpr int kAuxBytes = 1024 + kGatherWarps * NT * 4;
-    static constexpr int kStagingBytes = 2 * 2 * kStageRows * kStageRowBytes;  // 2 groups x 2 bufs
-    static constexpr int kStagesRaw =
-        (kMaxSmem - 1024 - kAuxBytes - kStagingBytes) / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kAccCols = 2 * NT;                        // per accumulator buffer
-    static constexpr int kNBufRaw = 512 / kAccCols;                // accumulators in flight
-    static constexpr int kNBuf = kNBufRaw > 8 ? 8 : kNBufRaw;
-    static constexpr int kUsedCols = kAccCols * kNBuf;
-    static constexpr int kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64
-                                   : kUsedCols <= 128 ? 128 : kUsedCols <= 256 ? 256 : 512;
-    static constexpr uint32_t kTxBytes = kNA * kATileBytes + (MODE == 1 ? kBTileBytes : 0);
-    // shared memory: 1 KB alignment slack + ring + barriers/aux
-    // Gather groups.  A waiter on a ring slot's mbarrier must never be more than one
-    // phase ahead of it (a parity wait cannot tell phase n from n - 2); group g
-    // handles stages g, g + G, ..., so G <= kStages guarantees it.  The W warps of
-    // a group split the rows of its stages.
-    static constexpr int kG = kGatherWarps < kStages ? kGatherWarps : kStages;
-    static constexpr int kW = kGatherWarps / kG;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kStagingBytes + kAuxBytes;
-    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N tile");
-    static_assert(kStages >= 2, "pipeline depth");
-    static_assert(kStageBytes % 1024 == 0, "stage alignment");
-};
-
-struct Aux {
-    uint64_t full[16];
-    uint64_t empty[16];
-    uint64_t tfull[8];
-    uint64_t tempty[8];
-    uint64_t drain;
-    uint32_t tmem_base;
-    int abort;
-    int last;
-    int pad;
-};
-
-__device__ __forceinline__ int split_count(const FfnArgs& a, int ntiles)
-{
-    // enough (tile, feature block, slice) units for ~16 waves of CTAs, each slice
-    // at least min_kt_per_split K tiles long
-    const int units = ntiles * a.fb_count;
-    if (units <= 0) return 1;
-    int s = (16 * (int)gridDim.x + units - 1) / units;
-    s = min(s, a.s_max);
-    s = min(s, max(1, a.num_kt / a.min_kt_per_split));
-    return max(s, 1);
-}
-
-// silu(g) * u = g * u / (1 + e^-g).  The result is rounded to bf16 (8-bit
-// significand), so the fast exponential and reciprocal (a few ulp of fp32) are
-// far inside that rounding; for g -> -inf the reciprocal of inf is 0.
-__device__ __forceinline__ float silu_mul(float g, float u)
-{
-    return g * __frcp_rn(1.0f + __expf(-g)) * u;
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int n)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// bar.red.or over `n` threads: true in every thread if any thread passed true.
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
-
-// Tile list entries are read through L2 (they may be read before this grid's
-// dependency wait; see the kernel).
-__device__ __forceinline__ Tile load_tile(const Tile* p)
-{
-    const int4 lo = __ldcg(reinterpret_cast<const int4*>(p));
-    const int4 hi = __ldcg(reinterpret_cast<const int4*>(p) + 1);
-    Tile t;
-    t.expert = lo.x;
-    t.row_start = lo.y;
-    t.rows = lo.z;
-    t.first = lo.w;
-    t.count = hi.x;
-    t.pad[0] = hi.y;
-    t.pad[1] = hi.z;
-    t.pad[2] = hi.w;
-    return t;
-}
 
 __device__ __forceinline__ void flag_error(const FfnArgs& a, Aux* aux)
 {
@@ -252,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();
 
     const int ntiles = __ldcg(a.num_tiles);
-    const int s_want = split_count(a, ntiles);
+    const int s_want = split_count(ntiles * a.fb_count, a.s_max, a.num_kt, a.min_kt_per_split);
     const int kt_per_split = (a.num_kt + s_want - 1) / s_want;
     const int S = (a.num_kt + kt_per_split - 1) / kt_per_split;  // every slice non-empty
     const int units = ntiles * a.fb_count * S;
@@ -576,42 +465,6 @@ teardown:
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2D bf16 row-major [rows, cols] tensor map with a [box_rows, 64] box, 128-byte swizzle.
-cudaError_t make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                      uint32_t box_rows)
-{
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
 
 template <int MODE, int NT>
 cudaError_t launch_mode(const CUtensorMap& tw, const CUtensorMap& ta, const FfnArgs& a, int grid,

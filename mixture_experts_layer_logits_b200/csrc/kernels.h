@@ -92,6 +92,31 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
                                const FfnPlan& plan, cudaStream_t st,
                                cudaEvent_t between_gemms = nullptr, bool reduce_y = true);
 
+// w13 + SwiGLU, w2 and the combine in one persistent launch (fused_ffn.cu), for
+// weight-streaming shapes: at most 64 tokens, so every expert's rows fit one tile.
+struct FusedBuffers {
+    const void* x;
+    const void* w13;
+    const void* w2;
+    const int32_t* permuted_rows;
+    const Tile* tiles;
+    const int32_t* num_tiles;
+    const float* topk_weights;
+    void* act;         // bf16 [I / 64, R, 64] (K-blocked)
+    float* part2;      // fp32 [s2_max, R, H]
+    void* y;           // bf16 [R, H]
+    void* out;         // bf16 [T, H]
+    int32_t* counters; // [fused_ffn_counters()], zeroed by the permutation kernel
+    int32_t* splits;   // [2]
+    int32_t* err;
+};
+bool fused_ffn_eligible(int T, int E, int k, int H, int I, const FfnPlan& plan);
+int fused_ffn_counters(int T, int H, const FfnPlan& plan);
+cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, int I,
+                             const FfnPlan& plan, cudaStream_t st);
+// moe_forward uses the fused launch where eligible unless MOE_DISABLE_FUSED=1.
+bool fused_enabled();
+
 // out[t] = sum_j w[t,j] * y[t*k+j] (k <= 16).
 cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
                            cudaStream_t st);

@@ -22,6 +22,15 @@ bool pdl_enabled()
     return on;
 }
 
+bool fused_enabled()
+{
+    static const bool on = [] {
+        const char* v = getenv("MOE_DISABLE_FUSED");
+        return !(v && v[0] && v[0] != '0');
+    }();
+    return on;
+}
+
 namespace {
 thread_local int g_last_cuda_error = 0;
 }  // namespace
@@ -66,9 +75,11 @@ bool combine_shape_ok(const moe_shape_t& s)
 
 struct Layout {
     size_t err, ids, weights, offsets, rows, tiles, num_tiles, splits, chunks, partials, act, y,
-        total;
+        partials2, counters, total;
     FfnPlan plan;
     bool ffn;
+    bool fused;      // the shape qualifies for the one-launch FFN + combine
+    int n_counters;  // its arrival counters (zeroed by the permutation kernel)
 };
 
 Layout layout_for(const moe_shape_t& s)
@@ -101,6 +112,13 @@ Layout layout_for(const moe_shape_t& s)
         const size_t act_rows = R > (size_t)L.plan.nt ? R : (size_t)L.plan.nt;
         L.act = take(act_rows * I * 2);
         L.y = take(R * H * 2);
+        // the fused launch keeps w13's and w2's slices live at once
+        L.fused = fused_ffn_eligible(s.T, s.E, s.top_k, H, I, L.plan);
+        if (L.fused) {
+            L.partials2 = take(p2 * sizeof(float));
+            L.n_counters = fused_ffn_counters(s.T, H, L.plan);
+            L.counters = take((size_t)L.n_counters * sizeof(int32_t));
+        }
     }
     L.total = off;
     return L;
@@ -139,8 +157,8 @@ PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
     a.tiles = at<Tile>(ws, L.tiles);
     a.num_tiles = at<int32_t>(ws, L.num_tiles);
     a.nt = L.plan.nt;
-    a.counters = nullptr;
-    a.n_counters = 0;
+    a.counters = L.fused ? at<int32_t>(ws, L.counters) : nullptr;
+    a.n_counters = L.fused ? L.n_counters : 0;
     a.chunk_counts = at<int32_t>(ws, L.chunks);
     (void)s;
     return a;
@@ -287,6 +305,31 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
     moe_status_t r = mark(0);
     if (r == MOE_OK) r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st);
     if (r == MOE_OK) r = mark(1);
+    if (L.fused && fused_enabled()) {
+        // one launch: w13, w2 and the combine (the stage events in between all
+        // mark its end)
+        FusedBuffers b;
+        b.x = x;
+        b.w13 = w13;
+        b.w2 = w2;
+        b.permuted_rows = rows;
+        b.tiles = at<Tile>(ws, L.tiles);
+        b.num_tiles = at<int32_t>(ws, L.num_tiles);
+        b.topk_weights = wts;
+        b.act = at<void>(ws, L.act);
+        b.part2 = at<float>(ws, L.partials2);
+        b.y = y;
+        b.out = out;
+        b.counters = at<int32_t>(ws, L.counters);
+        b.splits = at<int32_t>(ws, L.splits);
+        b.err = at<int32_t>(ws, L.err);
+        FfnPlan plan = L.plan;
+        plan.grid = device_sms();
+        if (r == MOE_OK)
+            r = cuda_status(launch_fused_ffn(b, s.T, s.E, s.top_k, s.H, s.I, plan, st));
+        for (int i = 2; i <= 4 && r == MOE_OK; ++i) r = mark(i);
+        return r;
+    }
     // a split w2 is reduced inside the combine (one launch fewer)
     const bool split2 = L.plan.s2_max > 1;
     if (r == MOE_OK)
@@ -328,8 +371,15 @@ int moe_forward_kernel_count(moe_shape_t s)
     if (!ffn_shape_ok(s)) return 0;
     const long R = (long)s.T * s.top_k;
     const Layout L = layout_for(s);
+    if (L.fused && fused_enabled()) return (R <= kSmallRows ? 1 : 3) + 1;
     // route(+permute) kernels, w13, [SwiGLU finalize], w2, combine
     return (R <= kSmallRows ? 1 : 3) + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
+}
+
+int moe_forward_fused(moe_shape_t s)
+{
+    if (!ffn_shape_ok(s)) return 0;
+    return layout_for(s).fused && fused_enabled() ? 1 : 0;
 }
 
 moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream)

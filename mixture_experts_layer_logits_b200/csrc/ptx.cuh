@@ -33,6 +33,32 @@ __device__ __forceinline__ void pdl_launch_dependents()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- cross-CTA flags
+
+// Load with acquire semantics at GPU scope: the loads this thread issues after it
+// observe everything the releasing thread (fence + atomic) published before.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Add with release semantics at GPU scope, no value returned: everything this
+// thread wrote -- and, through a preceding barrier, what the threads it
+// synchronised with wrote -- is visible before the increment is.
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy global accesses with its async-proxy ones
+// (TMA) on either side of the fence.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

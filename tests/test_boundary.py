@@ -165,3 +165,16 @@ def test_product_package_does_not_reference_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "moe_oracle" not in text and "libmoe_oracle" not in text, f
+
+
+def test_fused_forward_selection(lib):
+    """moe_forward runs FFN + combine as one launch exactly for T <= 64 shapes."""
+    if os.environ.get("MOE_DISABLE_FUSED", "0") not in ("", "0"):
+        pytest.skip("MOE_DISABLE_FUSED is set")
+    assert lib.moe_forward_fused(S()) == 1                              # decode, T = 8
+    assert lib.moe_forward_fused(S(T=64, E=256, H=7168, I=2048)) == 1   # skewed decode
+    assert lib.moe_forward_fused(S(T=65)) == 0
+    assert lib.moe_forward_fused(S(T=8192, H=4096, I=1536)) == 0        # prefill
+    assert lib.moe_forward_fused(S(H=100)) == 0                         # unsupported shape
+    assert lib.moe_forward_kernel_count(S()) == 2
+    assert lib.moe_forward_kernel_count(S(T=65)) >= 4

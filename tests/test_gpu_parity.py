@@ -248,3 +248,71 @@ def test_forward_without_pdl_is_identical(tmp_path):
         subprocess.run([sys.executable, str(script), str(path)], env=env, check=True, timeout=600)
         outs.append(torch.load(path))
     assert torch.equal(outs[0], outs[1])
+
+
+# Shapes for the one-launch FFN + combine (T <= 64): both w2 split choices,
+# the multi-launch path's w13 split both on (H >= 512) and off, an odd number
+# of 128-row w2 blocks, k = 16 over 1024 experts, one token.
+FUSED_SHAPES = [
+    ("tiny", None),
+    ("decode", None),
+    ("skewed_decode", None),
+    ("w13_split_only", (8, 16, 2, 1024, 256, 0.0)),
+    ("odd_w2_blocks", (8, 32, 4, 384, 256, 0.0)),
+    ("many_experts", (40, 1024, 16, 128, 128, 0.0)),
+    ("one_token", (1, 4, 2, 256, 128, 0.0)),
+]
+
+
+def _fused_workload(name, spec):
+    if spec is None:
+        return wl.WORKLOADS[name]
+    T, E, k, H, I, z = spec
+    return wl.custom(name, T, E, k, H, I, zipf_s=z)
+
+
+def test_fused_launch_against_multi_launch_and_oracle(tmp_path):
+    """moe_forward's one-launch path (T <= 64) against the multi-launch path
+    (MOE_DISABLE_FUSED=1, in a subprocess) and against the oracle.
+
+    Routing outputs are identical.  The one-launch path runs w13 unsplit, so out
+    is bit-identical to the multi-launch path wherever that path does too (its
+    w13 split needs H >= 512), and otherwise within the parity tolerance."""
+    script = tmp_path / "unfused.py"
+    script.write_text(
+        "import sys, torch\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        f"sys.path.insert(0, {os.path.join(ROOT, 'tests')!r})\n"
+        "import mixture_experts_layer_logits_b200 as moe\n"
+        "from test_gpu_parity import FUSED_SHAPES, _fused_workload\n"
+        "from mixture_experts_layer_logits_b200 import workloads as wl\n"
+        "res = {}\n"
+        "for name, spec in FUSED_SHAPES:\n"
+        "    w = _fused_workload(name, spec)\n"
+        "    d = wl.make_inputs(w, seed=13, device='cuda')\n"
+        "    assert not moe.moe_forward_fused(w.T, w.E, w.k, w.H, w.I)\n"
+        "    res[name] = moe.moe_forward(d['x'], d['logits'], d['w13'], d['w2'], w.k).cpu()\n"
+        "torch.save(res, sys.argv[1])\n")
+    path = tmp_path / "unfused.pt"
+    env = dict(os.environ, MOE_DISABLE_FUSED="1")
+    subprocess.run([sys.executable, str(script), str(path)], env=env, check=True, timeout=900)
+    ref = torch.load(path)
+    for name, spec in FUSED_SHAPES:
+        w = _fused_workload(name, spec)
+        d = wl.make_inputs(w, seed=13, device="cuda")
+        assert moe.moe_forward_fused(w.T, w.E, w.k, w.H, w.I), name
+        assert moe.moe_forward_kernel_count(w.T, w.E, w.k, w.H, w.I) == 2, name
+        out, ids, wts, off, rows = run_forward(w, d)
+        multi = ref[name]
+        if w.H < 512:
+            assert torch.equal(out.cpu(), multi), name
+        else:
+            assert_out_close(out, multi.float().numpy().astype(np.float64), what=f"{name} vs multi-launch")
+        # the one-launch result against the oracle, on sampled tokens
+        ref_ids, ref_w = oracle.route(host_f32(d["logits"]), w.k)
+        assert_routing_equal(ids, wts, ref_ids, ref_w)
+        toks = sorted(set([0, w.T // 2, w.T - 1]))
+        w13s, w2s = expert_weights_for(toks, ref_ids, d["w13"], d["w2"])
+        want = oracle.forward_tokens(host_bits(d["x"]), host_f32(d["logits"]), w13s, w2s, w.k,
+                                     toks, w.I)
+        assert_out_close(out[toks], want, what=f"{name} out[{toks}]")
