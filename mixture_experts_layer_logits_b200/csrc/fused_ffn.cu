@@ -84,7 +84,14 @@ struct Unit {
     int tile;
     int fb;
     int kt0, kt1;
+    int expert, row_start, rows;  // of the tile
 };
+
+// Each CTA decodes its unit list once into shared memory (two dependent L2
+// loads per unit, all units at once) instead of once per unit in every role;
+// a single-threaded TMA producer would otherwise stall on them between units.
+constexpr int kUnitTable = 128;
+constexpr int kUnitTableBytes = kUnitTable * 32;
 
 // The combine's routing weights, in shared memory right after Aux.
 struct ComboScratch {
@@ -130,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Aux* aux = reinterpret_cast<Aux*>(staging + C::kStagingBytes);
     ComboScratch* combo = reinterpret_cast<ComboScratch*>(aux + 1);
     int* tok_off = reinterpret_cast<int*>(combo + 1);
+    int4* unit_tab = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(aux) + C::kAuxBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -220,6 +228,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         un.tile = probe.first + local % probe.count;
         un.kt0 = un.split * ktps;
         un.kt1 = min(nkt, un.kt0 + ktps);
+        const Tile t = load_tile(a.tiles + un.tile);
+        un.expert = t.expert;
+        un.row_start = t.row_start;
+        un.rows = t.rows;
+        return un;
+    };
+    for (int i = threadIdx.x; i < min(my_units, kUnitTable); i += blockDim.x) {
+        const Unit un = decode(unit_of(i));
+        unit_tab[2 * i] = make_int4(un.ph | (un.split << 8), un.tile, un.fb, un.kt0 | (un.kt1 << 16));
+        unit_tab[2 * i + 1] = make_int4(un.expert, un.row_start, un.rows, 0);
+    }
+    __syncthreads();
+    auto fetch = [&](int i) {  // the CTA's i-th unit
+        if (i >= kUnitTable) return decode(unit_of(i));
+        const int4 e0 = unit_tab[2 * i], e1 = unit_tab[2 * i + 1];
+        Unit un;
+        un.ph = e0.x & 0xff;
+        un.split = e0.x >> 8;
+        un.tile = e0.y;
+        un.fb = e0.z;
+        un.kt0 = e0.w & 0xffff;
+        un.kt1 = e0.w >> 16;
+        un.expert = e1.x;
+        un.row_start = e1.y;
+        un.rows = e1.z;
         return un;
     };
 
@@ -233,8 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
             bool ok = true;
             for (int i = 0; i < my_units && ok; ++i) {
-                const Unit un = decode(unit_of(i));
-                const Tile t = load_tile(a.tiles + un.tile);
+                const Unit un = fetch(i);
+                const Unit& t = un;
                 const CUtensorMap* tm = un.ph ? &tm_w2 : &tm_w13;
                 // w13: the gate block and the up block of feature block fb; w2: two
                 // consecutive 128-row blocks of w2[e] (the second may belong to the
@@ -276,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int lu = 0; lu < my_units && ok; ++lu) {
-                const Unit un = decode(unit_of(lu));
-                const Tile t = load_tile(a.tiles + un.tile);
+                const Unit un = fetch(lu);
+                const Unit& t = un;
                 const int b = lu % C::kNBuf;
                 const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
                 if (!mbar_wait(&aux->tempty[b], aphase ^ 1u, abort_flag)) {
@@ -329,13 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             int cur_tile = -1, cur_ph = -1, ready_tile = -1;
             bool ok = true;
             for (int i = 0; i < my_units && ok; ++i) {
-                const Unit un = decode(unit_of(i));
+                const Unit un = fetch(i);
                 // first stage of this unit that this warp's group owns
                 int kt = un.kt0 + ((g - q % G) + G) % G;
                 const int q_unit0 = q;
                 q += un.kt1 - un.kt0;
                 if (kt >= un.kt1) continue;
-                const Tile t = load_tile(a.tiles + un.tile);
+                const Unit& t = un;
                 if (un.ph == 1 && un.tile != ready_tile) {
                     // every w13 unit of this tile has stored its act rows or slices
                     if (!warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
@@ -408,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* gstage = staging + grp * 2 * (kStageRows * kStageRowBytes);
         int chunk = 0;  // staging chunks issued by this group (buffer parity)
         for (int lu = 0; lu < my_units; ++lu) {
-            const Unit un = decode(unit_of(lu));
-            const Tile t = load_tile(a.tiles + un.tile);
+            const Unit un = fetch(lu);
+            const Unit& t = un;
             const int b = lu % C::kNBuf;
             const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
             const bool got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
@@ -585,9 +618,12 @@ cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const
                             const FusedArgs& a, int grid, cudaStream_t st)
 {
     using C = Cfg<0, NT>;
-    // the combine's weights sit in the slack Cfg reserves next to Aux
+    // the combine's weights sit in the slack Cfg reserves next to Aux; the unit
+    // table follows the aux area
     static_assert(sizeof(Aux) + sizeof(ComboScratch) <= 1024, "aux area");
-    constexpr int smem = C::kSmemBytes;
+    static_assert(C::kAuxBytes % 16 == 0, "unit table alignment");
+    constexpr int smem = C::kSmemBytes + kUnitTableBytes;
+    static_assert(smem <= C::kMaxSmem, "shared memory");
     auto kern = fused_ffn_kernel<NT>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
