@@ -33,6 +33,14 @@ struct PermuteAux {
     int32_t* counters;     // split-K arrival counters to zero, [n_counters]
     int n_counters;
     int32_t* chunk_counts; // [n_chunks, E] scratch of the multi-CTA path
+    // L2 prefetch of w13 for the one-launch FFN (single-CTA path, with routing):
+    // the launch gets pf_units CTAs, and CTA b >= 1 prefetches the first pf_kt K
+    // tiles of the gate and up blocks of w13 unit b (fused CTA b's first unit)
+    // through the tensor map passed with the launch.  pf_units = 0: off.
+    int pf_units;
+    int pf_fb13;   // I / 128
+    int pf_I;
+    int pf_kt;
 };
 
 // Records the cudaError_t that moe_last_cuda_error() reports on this host thread.
@@ -49,7 +57,8 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids,
 constexpr int kSmallRows = 4096;
 cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k, int32_t* ids,
                                        float* weights, int32_t* offsets, int32_t* rows,
-                                       const PermuteAux& aux, cudaStream_t st);
+                                       const PermuteAux& aux, cudaStream_t st,
+                                       const CUtensorMap* pf_w13 = nullptr);
 
 // Multi-CTA path: per-chunk counts, then a per-chunk stable scatter whose CTAs
 // each scan the count table themselves (CTA 0 also writes offsets and tiles).

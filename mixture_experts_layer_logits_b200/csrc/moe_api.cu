@@ -8,6 +8,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include "gemm_common.cuh"
 #include "kernels.h"
 #include "moe.h"
 
@@ -160,20 +161,35 @@ PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
     a.counters = L.fused ? at<int32_t>(ws, L.counters) : nullptr;
     a.n_counters = L.fused ? L.n_counters : 0;
     a.chunk_counts = at<int32_t>(ws, L.chunks);
+    a.pf_units = 0;
+    a.pf_fb13 = a.pf_I = a.pf_kt = 0;
     (void)s;
     return a;
 }
 
+// w13_prefetch: for the one-launch FFN, the w13 weights whose first K tiles the
+// permutation kernel prefetches into L2 (single-CTA path only).
 moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, const moe_shape_t& s,
                          int32_t* offsets, int32_t* rows, void* ws, const Layout& L,
-                         cudaStream_t st)
+                         cudaStream_t st, const void* w13_prefetch = nullptr)
 {
-    const PermuteAux aux = make_aux(ws, L, s);
+    PermuteAux aux = make_aux(ws, L, s);
     const long R = (long)s.T * s.top_k;
     cudaError_t e;
     if (R <= kSmallRows) {
+        CUtensorMap pf;
+        const CUtensorMap* pf_map = nullptr;
+        if (w13_prefetch &&
+            gemm::make_tmap(&pf, w13_prefetch, (uint64_t)s.E * 2 * s.I, (uint64_t)s.H, gemm::kBM) ==
+                cudaSuccess) {
+            pf_map = &pf;
+            aux.pf_units = device_sms();  // the fused grid: each CTA's first w13 unit
+            aux.pf_fb13 = s.I / gemm::kBM;
+            aux.pf_I = s.I;
+            aux.pf_kt = s.H / gemm::kBK < 8 ? s.H / gemm::kBK : 8;
+        }
         e = launch_small_route_permute(logits, s.T, s.E, s.top_k, ids, weights, offsets, rows, aux,
-                                       st);
+                                       st, pf_map);
     } else {
         e = cudaSuccess;
         if (logits) e = launch_route(logits, s.T, s.E, s.top_k, ids, weights, st);
@@ -302,10 +318,11 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
         return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st));
     };
 
+    const bool fused = L.fused && fused_enabled();
     moe_status_t r = mark(0);
-    if (r == MOE_OK) r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st);
+    if (r == MOE_OK) r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st, fused ? w13 : nullptr);
     if (r == MOE_OK) r = mark(1);
-    if (L.fused && fused_enabled()) {
+    if (fused) {
         // one launch: w13, w2 and the combine (the stage events in between all
         // mark its end)
         FusedBuffers b;

@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "kernels.h"
 #include "ptx.cuh"
@@ -212,8 +213,10 @@ __device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, in
     for (int off = 1; off < 16; off <<= 1) sum += __shfl_xor_sync(kFull, sum, off);
     sum = __shfl_sync(kFull, sum, 0);
     if (lane < k) {
-        ids[lane] = my_id;
-        weights[lane] = ex / sum;
+        if (ids) {
+            ids[lane] = my_id;
+            weights[lane] = ex / sum;
+        }
         if (ids_s) ids_s[lane] = my_id;
     }
 }
@@ -350,15 +353,56 @@ __global__ void __launch_bounds__(256, 4) route_kernel(const float* __restrict__
 }
 
 // One CTA: (route) + count + scan + stable scatter + tile list, for T*k <= kSmallRows.
+// CTAs 1.. of the single-CTA permutation launch when the one-launch FFN follows
+// (aux.pf_units > 0).  Each routes the T tokens again (ids into shared memory
+// only; CTA 0 writes every output), ranks the touched experts -- with T no
+// larger than the tile height every expert's rows form one tile, so tile j is
+// the j-th touched expert -- and prefetches into L2 the first pf_kt K tiles of
+// the gate and up blocks of w13 unit blockIdx.x: the first unit of fused CTA
+// blockIdx.x (tile = unit / fb13, feature block = unit % fb13).  Spread over the
+// grid, the weight stream starts while CTA 0 is still permuting; from one SM
+// the prefetches would drain at a single TMA unit's rate.  A hint only.
+template <int V, bool VEC>
+__device__ __forceinline__ void prefetch_first_unit(const float* __restrict__ logits, int T, int E,
+                                                    int k, const PermuteAux& aux,
+                                                    const CUtensorMap* w13, int* flag,
+                                                    int (*sel)[16], float2 (*cand)[32], int* sums)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) flag[e] = 0;
+    __syncthreads();
+    for (int t = warp; t < T; t += 32) {
+        float v[V];
+        warp_load_row<V, VEC>(logits + (size_t)t * E, E, lane, v);
+        warp_select_token<V, VEC>(v, E, k, lane, nullptr, nullptr, sel[warp], cand[warp]);
+        __syncwarp();
+        if (lane < k) flag[sel[warp][lane]] = 1;
+        __syncwarp();
+    }
+    __syncthreads();
+    const int e = threadIdx.x;
+    const int touched = e < E ? flag[e] : 0;
+    int total;
+    const int rank = block_exclusive_scan(touched, sums, total);  // ends with a barrier
+    if (touched) flag[rank] = e;  // flag[j] = expert of tile j
+    __syncthreads();
+    const int tile = blockIdx.x / aux.pf_fb13, fb = blockIdx.x % aux.pf_fb13;
+    if (tile < total && threadIdx.x < 2 * aux.pf_kt) {
+        const int half = threadIdx.x / aux.pf_kt, kt = threadIdx.x % aux.pf_kt;
+        tma_prefetch_l2_2d(w13, kt * 64, flag[tile] * 2 * aux.pf_I + half * aux.pf_I + fb * 128);
+    }
+}
+
 template <int V, bool VEC>
 __global__ void __launch_bounds__(1024, 1)
     small_route_permute_kernel(const float* __restrict__ logits, int T, int E, int k,
                                int32_t* __restrict__ ids, float* __restrict__ weights,
                                int32_t* __restrict__ offsets, int32_t* __restrict__ rows_out,
-                               PermuteAux aux)
+                               PermuteAux aux, const __grid_constant__ CUtensorMap pf_w13)
 {
     extern __shared__ int smem[];
     __shared__ int sums[32];
+    __shared__ float2 cand[32][32];
     const int R = T * k;
     int* ids_s = smem;
     int* table = smem + ((R + 3) & ~3);
@@ -367,8 +411,12 @@ __global__ void __launch_bounds__(1024, 1)
     pdl_wait();
     pdl_launch_dependents();
 
+    if (blockIdx.x > 0) {  // L2 prefetch CTAs (launched only with logits and aux.pf_units)
+        __shared__ int sel[32][16];
+        prefetch_first_unit<V, VEC>(logits, T, E, k, aux, &pf_w13, smem, sel, cand, sums);
+        return;
+    }
     if (logits) {
-        __shared__ float2 cand[32][32];
         // a warp's next token is loaded while its current one is selected
         float v[V];
         if (warp < T) warp_load_row<V, VEC>(logits + (size_t)warp * E, E, lane, v);
@@ -559,27 +607,34 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids,
 template <int V, bool VEC>
 static cudaError_t launch_small_v(const float* logits, int T, int E, int k, int32_t* ids,
                                   float* weights, int32_t* offsets, int32_t* rows,
-                                  const PermuteAux& aux, cudaStream_t st)
+                                  const PermuteAux& aux, cudaStream_t st, const CUtensorMap& pf)
 {
     const int R = T * k;
-    const size_t smem = sizeof(int) * (size_t)(((R + 3) & ~3) + 32 * E);
+    const size_t smem = sizeof(int) * (size_t)(((R + 3) & ~3) + 32 * E);  // >= E ints
     cudaError_t err = cudaFuncSetAttribute(small_route_permute_kernel<V, VEC>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    return launch(small_route_permute_kernel<V, VEC>, dim3(1), dim3(1024), smem, st, logits, T, E,
-                  k, ids, weights, offsets, rows, aux);
+    const int grid = (logits && aux.pf_units > 1) ? aux.pf_units : 1;  // CTAs 1.. prefetch
+    return launch(small_route_permute_kernel<V, VEC>, dim3(grid), dim3(1024), smem, st, logits, T,
+                  E, k, ids, weights, offsets, rows, aux, pf);
 }
 
 cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k, int32_t* ids,
                                        float* weights, int32_t* offsets, int32_t* rows,
-                                       const PermuteAux& aux, cudaStream_t st)
+                                       const PermuteAux& aux, cudaStream_t st,
+                                       const CUtensorMap* pf_w13)
 {
     const bool vec = (E % 4) == 0;
+    CUtensorMap none;
+    memset(&none, 0, sizeof(none));  // never read: pf_units == 0 without a map
+    PermuteAux a = aux;
+    if (!pf_w13) a.pf_units = 0;
+    const CUtensorMap& pf = pf_w13 ? *pf_w13 : none;
 #define MOE_SMALL(V)                                                                              \
     (vec && (V) >= 4 ? launch_small_v<V, ((V) >= 4)>(logits, T, E, k, ids, weights, offsets, rows, \
-                                                     aux, st)                                     \
-                     : launch_small_v<V, false>(logits, T, E, k, ids, weights, offsets, rows, aux, \
-                                                st))
+                                                     a, st, pf)                                   \
+                     : launch_small_v<V, false>(logits, T, E, k, ids, weights, offsets, rows, a,   \
+                                                st, pf))
     switch (logits ? values_per_lane(E) : 1) {
     case 1: return MOE_SMALL(1);
     case 2: return MOE_SMALL(2);
