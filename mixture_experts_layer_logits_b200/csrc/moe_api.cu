@@ -186,7 +186,11 @@ moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, cons
             aux.pf_units = device_sms();  // the fused grid: each CTA's first w13 unit
             aux.pf_fb13 = s.I / gemm::kBM;
             aux.pf_I = s.I;
-            aux.pf_kt = s.H / gemm::kBK < 8 ? s.H / gemm::kBK : 8;
+            // 16 K tiles (2 x 128 x 1024 weights per CTA) cover the routing and
+            // fused-kernel set-up window; 8 left HBM idle part of it, 20 and 24
+            // gained nothing more (same-B200 A/B)
+            constexpr int kPrefetchKt = 16;
+            aux.pf_kt = s.H / gemm::kBK < kPrefetchKt ? s.H / gemm::kBK : kPrefetchKt;
         }
         e = launch_small_route_permute(logits, s.T, s.E, s.top_k, ids, weights, offsets, rows, aux,
                                        st, pf_map);
