@@ -69,6 +69,7 @@ struct FusedArgs {
     __nv_bfloat16* out;           // [T, H]
     int32_t* tile_ready;          // [max_tiles] w13 arrivals, zero at entry
     int32_t* token_ready;         // [T * fb2] w2 row arrivals, zero at entry
+    int32_t* w2_next;             // w2 units handed out at run time, zero at entry
     int32_t* split_out;           // [2] 1, S2 (CTA 0)
     int32_t* err;
     int k, H, I, R;
@@ -87,11 +88,15 @@ struct Unit {
     int expert, row_start, rows;  // of the tile
 };
 
-// Each CTA decodes its unit list once into shared memory (two dependent L2
-// loads per unit, all units at once) instead of once per unit in every role;
-// a single-threaded TMA producer would otherwise stall on them between units.
+// Each CTA keeps its unit list in shared memory: the static part decoded once
+// (two dependent L2 loads per unit, all units at once) instead of once per unit
+// in every role -- a single-threaded TMA producer would otherwise stall on them
+// between units -- and the dynamic part published by the producer as it claims
+// units.  32 bytes per entry plus a sequence word.
 constexpr int kUnitTable = 128;
-constexpr int kUnitTableBytes = kUnitTable * 32;
+constexpr int kUnitTableBytes = kUnitTable * (32 + 4);
+constexpr int kUnitEnd = 2;    // Unit::ph of the list's terminator
+constexpr int kUnitAbort = 3;  // Unit::ph when waiting for an entry gave up
 
 // The combine's routing weights, in shared memory right after Aux.
 struct ComboScratch {
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ComboScratch* combo = reinterpret_cast<ComboScratch*>(aux + 1);
     int* tok_off = reinterpret_cast<int*>(combo + 1);
     int4* unit_tab = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(aux) + C::kAuxBytes);
+    int* tab_seq = reinterpret_cast<int*>(unit_tab + 2 * kUnitTable);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -190,25 +196,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     volatile int* abort_flag = &aux->abort;
 
-    // Static schedule, the same in every role.  CTA b runs w13 units b, b + G, ...
-    // When U13 is not a multiple of G, the CTAs with one unit fewer ("light",
-    // b >= U13 % G) next take `fill` w2 units each -- about one w13 unit's worth of
-    // K tiles, the lowest w2 indices -- and the w2 units left are dealt round-robin.
-    // Each CTA's list is its w13 units, then its w2 units in increasing order.
+    // Schedule.  CTA b first runs w13 units b, b + G, ...  When U13 is not a
+    // multiple of G, the CTAs with one unit fewer ("light", b >= U13 % G) next
+    // take `fill` w2 units each -- about one w13 unit's worth of K tiles, the
+    // lowest w2 indices.  Those lists are static.  The w2 units left are handed
+    // out in increasing order at run time: a CTA's producer claims the next one
+    // with an atomic on a workspace counter when it is ready for more, so CTAs
+    // that stream faster take more and all of them finish together.
     const int G = gridDim.x, bid = blockIdx.x;
     const int r13 = U13 % G;
     const int n13 = U13 / G + (bid < r13 ? 1 : 0);
     const int nlight = r13 ? G - r13 : 0;
     const int fill = nlight ? min((a.kt13 + ktps2 / 2) / ktps2, U2 / nlight) : 0;
     const int nf = (nlight && bid >= r13) ? fill : 0;
-    const int rest0 = nlight * fill;
-    const int nrest = U2 - rest0 > bid ? (U2 - rest0 - bid + G - 1) / G : 0;
-    const int my_units = n13 + nf + nrest;
-    auto unit_of = [&](int i) {  // global unit: [0, U13) w13, [U13, U13 + U2) w2
-        if (i < n13) return bid + i * G;
-        i -= n13;
-        if (i < nf) return U13 + (bid - r13) + i * nlight;
-        return U13 + rest0 + bid + (i - nf) * G;
+    const int rest0 = nlight * fill;  // the first w2 unit handed out at run time
+    const int n_static = n13 + nf;
+    auto unit_of = [&](int i) {  // global unit of static entry i: [0, U13) w13, then w2
+        return i < n13 ? bid + i * G : U13 + (bid - r13) + (i - n13) * nlight;
     };
 
     // unit u -> (phase, slice, tile, feature block), each phase in grouped_ffn.cu's
@@ -234,15 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         un.rows = t.rows;
         return un;
     };
-    for (int i = threadIdx.x; i < min(my_units, kUnitTable); i += blockDim.x) {
-        const Unit un = decode(unit_of(i));
-        unit_tab[2 * i] = make_int4(un.ph | (un.split << 8), un.tile, un.fb, un.kt0 | (un.kt1 << 16));
-        unit_tab[2 * i + 1] = make_int4(un.expert, un.row_start, un.rows, 0);
-    }
-    __syncthreads();
-    auto fetch = [&](int i) {  // the CTA's i-th unit
-        if (i >= kUnitTable) return decode(unit_of(i));
-        const int4 e0 = unit_tab[2 * i], e1 = unit_tab[2 * i + 1];
+    auto put = [&](int slot, const Unit& un) {
+        unit_tab[2 * slot] = make_int4(un.ph | (un.split << 8), un.tile, un.fb, un.kt0 | (un.kt1 << 16));
+        unit_tab[2 * slot + 1] = make_int4(un.expert, un.row_start, un.rows, 0);
+    };
+    auto read = [&](int slot) {
+        const int4 e0 = unit_tab[2 * slot], e1 = unit_tab[2 * slot + 1];
         Unit un;
         un.ph = e0.x & 0xff;
         un.split = e0.x >> 8;
@@ -255,6 +256,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         un.rows = e1.z;
         return un;
     };
+    for (int i = threadIdx.x; i < kUnitTable; i += blockDim.x) tab_seq[i] = 0;
+    for (int i = threadIdx.x; i < min(n_static, kUnitTable); i += blockDim.x)
+        put(i, decode(unit_of(i)));
+    __syncthreads();
+    // The CTA's i-th unit.  Dynamic entries live in the table as a ring with
+    // tab_seq[slot] = i + 1 once published; no role trails the producer by more
+    // than kStages + kNBuf units, far below the ring's length.
+    auto get = [&](int i) {
+        if (i < n_static) return i < kUnitTable ? read(i) : decode(unit_of(i));
+        const int slot = i % kUnitTable;
+        const volatile int* sq = tab_seq + slot;
+        if (*sq != i + 1) {
+            const uint64_t t0 = globaltimer_ns();
+            while (*sq != i + 1) {
+                __nanosleep(32);
+                if (*abort_flag || globaltimer_ns() - t0 > 2000000000ull) {
+                    flag_error(a.err, aux);
+                    Unit un;
+                    un.ph = kUnitAbort;
+                    return un;
+                }
+            }
+        }
+        __threadfence_block();
+        return read(slot);
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -265,8 +292,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued[16];
             for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
             bool ok = true;
-            for (int i = 0; i < my_units && ok; ++i) {
-                const Unit un = fetch(i);
+            for (int i = 0; ok; ++i) {
+                Unit un;
+                if (i < n_static) {
+                    un = get(i);
+                } else {  // claim the next w2 unit and publish it to the other roles
+                    const int v = rest0 + atomicAdd(a.w2_next, 1);
+                    if (v < U2) {
+                        un = decode(U13 + v);
+                    } else {
+                        un.ph = kUnitEnd;
+                        un.split = un.tile = un.fb = un.kt0 = un.kt1 = 0;
+                        un.expert = un.row_start = un.rows = 0;
+                    }
+                    put(i % kUnitTable, un);
+                    __threadfence_block();
+                    *reinterpret_cast<volatile int*>(tab_seq + i % kUnitTable) = i + 1;
+                    if (un.ph == kUnitEnd) break;
+                }
                 const Unit& t = un;
                 const CUtensorMap* tm = un.ph ? &tm_w2 : &tm_w13;
                 // w13: the gate block and the up block of feature block fb; w2: two
@@ -308,8 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int lu = 0; lu < my_units && ok; ++lu) {
-                const Unit un = fetch(lu);
+            for (int lu = 0; ok; ++lu) {
+                const Unit un = get(lu);
+                if (un.ph >= kUnitEnd) break;
                 const Unit& t = un;
                 const int b = lu % C::kNBuf;
                 const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
@@ -361,8 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int q = 0;  // global stage sequence number (same as the producer's)
             int cur_tile = -1, cur_ph = -1, ready_tile = -1;
             bool ok = true;
-            for (int i = 0; i < my_units && ok; ++i) {
-                const Unit un = fetch(i);
+            for (int i = 0; ok; ++i) {
+                const Unit un = get(i);
+                if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
                 // first stage of this unit that this warp's group owns
                 int kt = un.kt0 + ((g - q % G) + G) % G;
                 const int q_unit0 = q;
@@ -440,14 +485,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f_local = qw * 32 + lane;       // feature inside the 128-row block
         uint8_t* gstage = staging + grp * 2 * (kStageRows * kStageRowBytes);
         int chunk = 0;  // staging chunks issued by this group (buffer parity)
-        for (int lu = 0; lu < my_units; ++lu) {
-            const Unit un = fetch(lu);
+        for (int lu = 0;; ++lu) {
+            const Unit un = get(lu);
             const Unit& t = un;
             const int b = lu % C::kNBuf;
             const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
-            const bool got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
-            if (!got) flag_error(a.err, aux);
-            if (named_bar_or(1 + grp, 128, !got || *abort_flag)) break;  // same in all 4 warps
+            bool got = false;
+            if (un.ph < kUnitEnd) {
+                got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
+                if (!got) flag_error(a.err, aux);
+            }
+            // the end of the list, or a failure: the same decision in all 4 warps
+            if (named_bar_or(1 + grp, 128, un.ph >= kUnitEnd || !got || *abort_flag)) break;
             tc_fence_after();
             const int ph = un.ph;
             const int S = ph ? S2 : 1;
@@ -652,7 +701,7 @@ bool fused_ffn_eligible(int T, int E, int k, int H, int I, const FfnPlan& plan)
 
 int fused_ffn_counters(int T, int H, const FfnPlan& plan)
 {
-    return plan.max_tiles + T * ((H / kBM + 1) / 2);
+    return plan.max_tiles + T * ((H / kBM + 1) / 2) + 1;
 }
 
 cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, int I,
@@ -678,6 +727,7 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     a.out = static_cast<__nv_bfloat16*>(b.out);
     a.tile_ready = b.counters;
     a.token_ready = b.counters + plan.max_tiles;
+    a.w2_next = a.token_ready + (size_t)T * ((H / kBM + 1) / 2);
     a.split_out = b.splits;
     a.err = b.err;
     a.k = k;
