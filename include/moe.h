@@ -116,10 +116,12 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
  * are optional outputs: pass NULL to keep them inside the workspace.
  * For weight-streaming shapes (T <= 64, see moe_forward_fused) w13, w2 and the
  * combine run as ONE persistent launch whose CTAs hand act rows and finished y
- * rows to each other through arrival counters in the workspace; its result is
- * bit-identical to the multi-launch path, which MOE_DISABLE_FUSED=1 in the
- * environment selects instead.  Either way every wait is bounded (2 s; then
- * moe_device_status reports MOE_ERR_DEVICE_TIMEOUT). */
+ * rows to each other through arrival counters in the workspace.  It sums w13
+ * over the whole K range in one fp32 chain, so its result equals the
+ * multi-launch path's (MOE_DISABLE_FUSED=1 in the environment selects that
+ * path) bit for bit where that path leaves w13 unsplit (H < 512), and up to
+ * bf16 rounding of the differently ordered sum otherwise.  Either way every
+ * wait is bounded (2 s; then moe_device_status reports MOE_ERR_DEVICE_TIMEOUT). */
 moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
                          const moe_bf16_t* w2, moe_shape_t shape, moe_bf16_t* out,
                          int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
@@ -167,6 +169,18 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
 
 /* Number of kernels one moe_forward call launches for `shape` (0 if unsupported). */
 int moe_forward_kernel_count(moe_shape_t shape);
+
+/* Failure detection without a GPU fault.  Launches one small kernel whose two
+ * bounded waits cannot be satisfied -- an mbarrier that nothing arrives on and
+ * a workspace flag that nothing sets (workspace bytes [4, 8), zeroed first) --
+ * built from the same wait primitives as the layer's kernels.  Each gives up
+ * after limit_us microseconds and records the timeout in the workspace's error
+ * word exactly as a layer kernel does, so the next moe_device_status(workspace)
+ * returns MOE_ERR_DEVICE_TIMEOUT (and clears it); the CUDA context stays usable.
+ * workspace: device memory of at least 8 bytes, 16-byte aligned.
+ * limit_us: 1 .. 2,000,000, else MOE_ERR_INVALID_ARG. */
+moe_status_t moe_selftest_wait_timeout(void* workspace, size_t ws_bytes, unsigned limit_us,
+                                       moe_stream_t stream);
 
 /* 1 if moe_forward runs w13, w2 and the combine of `shape` as one persistent
  * launch (T <= 64 and T*k <= 4096, unless MOE_DISABLE_FUSED=1), else 0. */

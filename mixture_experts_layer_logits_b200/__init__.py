@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "MoeError", "Shape", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_forward_timed", "moe_forward_kernel_count",
-    "moe_forward_fused",
+    "moe_forward_fused", "moe_selftest_wait_timeout",
     "moe_device_status", "library_path", "load_library",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ERR_MISALIGNED",
     "MOE_ERR_WORKSPACE_TOO_SMALL", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
@@ -77,6 +77,9 @@ def load_library():
     lib.moe_forward_kernel_count.restype = ctypes.c_int
     lib.moe_forward_fused.argtypes = [Shape]
     lib.moe_forward_fused.restype = ctypes.c_int
+    lib.moe_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint,
+                                              ctypes.c_void_p]
+    lib.moe_selftest_wait_timeout.restype = ctypes.c_int
     lib.moe_device_status.argtypes = [_vp, ctypes.c_size_t, _vp]
     for fn in (lib.moe_route, lib.moe_permute, lib.moe_grouped_ffn, lib.moe_combine,
                lib.moe_forward, lib.moe_forward_timed, lib.moe_device_status):
@@ -242,6 +245,13 @@ def moe_forward_kernel_count(T: int, E: int, top_k: int, H: int, I: int) -> int:
 def moe_forward_fused(T: int, E: int, top_k: int, H: int, I: int) -> bool:
     """True if moe_forward runs the FFN and the combine as one persistent launch."""
     return bool(load_library().moe_forward_fused(Shape(T, E, top_k, H, I)))
+
+
+def moe_selftest_wait_timeout(ws: torch.Tensor, limit_us: int) -> None:
+    """Queue the failure-detection self-test: two unsatisfiable bounded waits that
+    give up after limit_us and record a timeout in ws (see moe_device_status)."""
+    _check(load_library().moe_selftest_wait_timeout(_ptr(ws), ws.numel(), int(limit_us),
+                                                    _stream(ws)), "moe_selftest_wait_timeout")
 
 
 def moe_device_status(ws: torch.Tensor) -> int:

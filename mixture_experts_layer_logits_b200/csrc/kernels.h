@@ -126,6 +126,10 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
 // moe_forward uses the fused launch where eligible unless MOE_DISABLE_FUSED=1.
 bool fused_enabled();
 
+// Failure-detection self-test (selftest.cu): a kernel whose bounded waits give
+// up after limit_us and record the timeout in the error word at ws[0].
+cudaError_t launch_wait_timeout_selftest(void* ws, unsigned limit_us, cudaStream_t st);
+
 // out[t] = sum_j w[t,j] * y[t*k+j] (k <= 16).
 cudaError_t launch_combine(const void* y, const float* weights, int T, int k, int H, void* out,
                            cudaStream_t st);

@@ -420,6 +420,15 @@ moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream)
     return v == kDeviceErrorMagic ? MOE_ERR_DEVICE_TIMEOUT : MOE_OK;
 }
 
+moe_status_t moe_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned limit_us,
+                                       moe_stream_t stream)
+{
+    if (!ws || limit_us < 1 || limit_us > 2000000u) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(ws)) return MOE_ERR_MISALIGNED;
+    if (ws_bytes < 2 * sizeof(int32_t)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    return cuda_status(launch_wait_timeout_selftest(ws, limit_us, static_cast<cudaStream_t>(stream)));
+}
+
 const char* moe_status_string(moe_status_t status)
 {
     switch (status) {

@@ -178,3 +178,12 @@ def test_fused_forward_selection(lib):
     assert lib.moe_forward_fused(S(H=100)) == 0                         # unsupported shape
     assert lib.moe_forward_kernel_count(S()) == 2
     assert lib.moe_forward_kernel_count(S(T=65)) >= 4
+
+
+def test_selftest_wait_timeout_validation(lib):
+    f = lib.moe_selftest_wait_timeout
+    assert f(NUL, 64, 1000, NUL) == moe.MOE_ERR_INVALID_ARG
+    assert f(A, 64, 0, NUL) == moe.MOE_ERR_INVALID_ARG             # limit out of range
+    assert f(A, 64, 2000001, NUL) == moe.MOE_ERR_INVALID_ARG
+    assert f(MIS, 64, 1000, NUL) == moe.MOE_ERR_MISALIGNED
+    assert f(A, 4, 1000, NUL) == moe.MOE_ERR_WORKSPACE_TOO_SMALL   # needs the error word + a flag
