@@ -47,7 +47,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch of a kernel from an ncu capture, keyed by
 # (workload, kernel), from the summaries under profiles/.  An entry is removed
 # when its kernel changes, until it is captured again.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("decode", "fused_ffn"): 509_732_608 + 4_027_392,  # profiles/fused_ffn_decode.md
+}
 
 
 def parse_args(argv=None):
