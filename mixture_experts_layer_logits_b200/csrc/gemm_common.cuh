@@ -75,6 +75,22 @@ struct Aux {
     int pad;
 };
 
+// TMEM columns an epilogue group reads per tcgen05.ld: 16, or 8 when a group's
+// half of the token columns is narrower (NT = 16), so no load reaches past the
+// group's columns -- and past the allocation in the last accumulator buffer.
+template <int NT>
+constexpr int kEpiCols = NT / 2 >= 16 ? 16 : 8;
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N])
+{
+    static_assert(N == 8 || N == 16, "tcgen05.ld width");
+    if constexpr (N == 16)
+        tmem_ld16(taddr, r);
+    else
+        tmem_ld8(taddr, r);
+}
+
 // Split-K slices wanted for `units` (tile, feature block) pairs: enough
 // (tile, feature block, slice) units for ~16 waves of CTAs, each slice at least
 // min_kt K tiles long.

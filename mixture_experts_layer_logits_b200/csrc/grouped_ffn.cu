@@ -425,13 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 continue;
             }
-            for (int j0 = jbeg; j0 < jend; j0 += 16) {
-                uint32_t g[16], v[16];
-                tmem_ld16(tacc + j0, g);
-                tmem_ld16(tacc + NT + j0, v);
+            constexpr int kCols = kEpiCols<NT>;
+            for (int j0 = jbeg; j0 < jend; j0 += kCols) {
+                uint32_t g[kCols], v[kCols];
+                tmem_ld_cols(tacc + j0, g);
+                tmem_ld_cols(tacc + NT + j0, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
+                for (int jj = 0; jj < kCols; ++jj) {
                     const int j = j0 + jj;
                     if (j >= jend) break;
                     const int p = t.row_start + j;
