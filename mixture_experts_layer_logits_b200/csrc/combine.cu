@@ -31,6 +31,7 @@ constexpr int kMaxSplits = 8;
 
 // One thread per (token, 8 hidden elements): the k rows are all loaded before
 // any is used, so a thread keeps up to 16 loads in flight.
+template <int KMAX>
 __global__ void __launch_bounds__(256)
     combine_kernel(const uint4* __restrict__ y, const float* __restrict__ w, int T, int k, int H8,
                    uint4* __restrict__ out)
@@ -40,10 +41,10 @@ __global__ void __launch_bounds__(256)
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long)T * H8) return;
     const int t = (int)(idx / H8), h8 = (int)(idx % H8);
-    uint4 v[kMaxK];
-    float wj[kMaxK];
+    uint4 v[KMAX];
+    float wj[KMAX];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         if (j < k) {
             const long r = (long)t * k + j;
             v[j] = __ldcs(y + r * H8 + h8);  // read once: stream
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         if (j < k) {  // j ascending: the fixed summation order
             const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
 #pragma unroll
@@ -225,8 +226,16 @@ cudaError_t launch_combine(const void* y, const float* weights, int T, int k, in
                            cudaStream_t st)
 {
     const int H8 = H / 8;
-    return launch_1d(combine_kernel, (long)T * H8, st, static_cast<const uint4*>(y), weights, T, k,
-                     H8, static_cast<uint4*>(out));
+    // the k rows' loads are unrolled up to a bound: registers for 16 rows would
+    // halve the resident threads at k = 8
+    auto go = [&](auto kern) {
+        return launch_1d(kern, (long)T * H8, st, static_cast<const uint4*>(y), weights, T, k, H8,
+                         static_cast<uint4*>(out));
+    };
+    if (k <= 2) return go(combine_kernel<2>);
+    if (k <= 4) return go(combine_kernel<4>);
+    if (k <= 8) return go(combine_kernel<8>);
+    return go(combine_kernel<kMaxK>);
 }
 
 cudaError_t launch_combine_partials(const float* partials, const int32_t* splits, const void* y,
