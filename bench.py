@@ -49,6 +49,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # when its kernel changes, until it is captured again.
 NCU_TRAFFIC = {
     ("decode", "fused_ffn"): 509_732_608 + 4_027_392,  # profiles/fused_ffn_decode.md
+    # profiles/grouped_gemm_prefill_shape.md: the 16-expert capture x 8
+    ("prefill", "w13"): 3_510_591_488,
+    ("prefill", "w2"): 2_175_619_072,
 }
 
 
