@@ -182,8 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int ntiles = __ldcg(a.num_tiles);
     // w13 is not split here: its epilogue writes bf16 act directly, which each w2
-    // stage then loads with one TMA.  w2 is split so the tail balances.
-    const int s2w = split_count(ntiles * a.fb2, a.s2_max, a.kt2, a.min_kt_per_split);
+    // stage then loads with one TMA.  w2 is split only as far as ~4 waves of units
+    // need: the run-time hand-out already balances the tail, and every extra
+    // slice adds epilogue publishes and combine reads (same-B200 A/B: 16 waves
+    // 101.4 us decode / 360.7 us skewed decode, 4 waves 98.2 / 341.8).
+    const int s2w = split_count(ntiles * a.fb2, a.s2_max, a.kt2, a.min_kt_per_split, 4);
     const int ktps2 = (a.kt2 + s2w - 1) / s2w;
     const int S2 = (a.kt2 + ktps2 - 1) / ktps2;  // every slice non-empty
     const int U13 = ntiles * a.fb13;

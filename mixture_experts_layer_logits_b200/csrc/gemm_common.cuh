@@ -92,12 +92,13 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N])
 }
 
 // Split-K slices wanted for `units` (tile, feature block) pairs: enough
-// (tile, feature block, slice) units for ~16 waves of CTAs, each slice at least
-// min_kt K tiles long.
-__device__ __forceinline__ int split_count(int units, int s_max, int num_kt, int min_kt)
+// (tile, feature block, slice) units for `waves` waves of CTAs, each slice at
+// least min_kt K tiles long.
+__device__ __forceinline__ int split_count(int units, int s_max, int num_kt, int min_kt,
+                                           int waves = 16)
 {
     if (units <= 0) return 1;
-    int s = (16 * (int)gridDim.x + units - 1) / units;
+    int s = (waves * (int)gridDim.x + units - 1) / units;
     s = min(s, s_max);
     s = min(s, max(1, num_kt / min_kt));
     return max(s, 1);
