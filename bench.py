@@ -138,6 +138,14 @@ def stage_work(w, n_touched):
     }
 
 
+def step_stats(step_ms, slowest):
+    """Median, p10 and p90 of the per-step event times (each the max over ranks)."""
+    q = statistics.quantiles(step_ms, n=10, method="inclusive") if len(step_ms) > 1 else \
+        [step_ms[0]] * 9
+    return {"median": round(slowest(statistics.median(step_ms)), 5),
+            "p10": round(slowest(q[0]), 5), "p90": round(slowest(q[8]), 5)}
+
+
 def roofline_entry(stage, work, ms, peaks, peak_kind, sustained, traffic):
     t = ms / 1e3
     hbm_t = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
@@ -369,7 +377,9 @@ def routing_bench(args, w, rank, world, local, dev, pg):
         torch.cuda.nvtx.range_pop()
         barrier()
         t_wall = time.perf_counter() - t_wall
-    ms = slowest(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    ms = slowest(statistics.mean(step_ms))
+    stats = step_stats(step_ms, slowest)
     route_ms = slowest(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
     perm_ms = slowest(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
 
@@ -418,7 +428,8 @@ def routing_bench(args, w, rank, world, local, dev, pg):
         line = {
             "metric": metric_name(w), "value": round(weak_scaling_value(world, T, ms), 2),
             "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(ms, 5), "ms_per_step_stats": stats,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
             "config": dict(w.as_dict(), parallelism=f"replicas{world}",
                            l2="flushed before every step (256 MiB write), outside the step events"),
@@ -533,6 +544,7 @@ def main(argv=None):
         t_wall = time.perf_counter() - t_wall
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = slowest(statistics.mean(step_ms))
+    stats = step_stats(step_ms, slowest)
     if moe.moe_device_status(ws) != moe.MOE_OK:
         raise SystemExit("device error during the timed steps")
 
@@ -608,6 +620,7 @@ def main(argv=None):
             "steps": K,
             "warmup": max(args.warmup, 3),
             "ms_per_step": round(ms, 5),
+            "ms_per_step_stats": stats,
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,

@@ -72,3 +72,14 @@ def test_single_rank_helpers():
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.rank_seed(0, 0) != bench.rank_seed(0, 1)
     assert bench.weak_scaling_value(1, 8, 0.125) == pytest.approx(64000.0)
+
+
+def test_step_stats():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    st = bench.step_stats([float(v) for v in range(1, 11)], lambda v: v)
+    assert st == {"median": 5.5, "p10": 1.9, "p90": 9.1}
+    assert bench.step_stats([0.25], lambda v: v) == {"median": 0.25, "p10": 0.25, "p90": 0.25}
+    # every statistic goes through the max-over-ranks reduction
+    assert bench.step_stats([1.0, 3.0], lambda v: v + 100)["median"] == 102.0
