@@ -252,7 +252,8 @@ def test_forward_without_pdl_is_identical(tmp_path):
 
 # Shapes for the one-launch FFN + combine (T <= 64): both w2 split choices,
 # the multi-launch path's w13 split both on (H >= 512) and off, an odd number
-# of 128-row w2 blocks, k = 16 over 1024 experts, one token.
+# of 128-row w2 blocks, k = 16 over 1024 experts, one token, the largest routed
+# row count (T * k = 1024, full 64-row tiles), and ragged 64-row tiles.
 FUSED_SHAPES = [
     ("tiny", None),
     ("decode", None),
@@ -261,6 +262,8 @@ FUSED_SHAPES = [
     ("odd_w2_blocks", (8, 32, 4, 384, 256, 0.0)),
     ("many_experts", (40, 1024, 16, 128, 128, 0.0)),
     ("one_token", (1, 4, 2, 256, 128, 0.0)),
+    ("full_tiles_k16", (64, 16, 16, 256, 256, 0.0)),   # T*k = 1024, every tile 64 rows
+    ("ragged_t33", (33, 64, 4, 512, 384, 0.0)),        # 64-row tiles, ragged; I / 128 = 3
 ]
 
 
