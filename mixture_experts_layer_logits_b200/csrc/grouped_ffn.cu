@@ -19,21 +19,21 @@
 //   warp 0      TMA producer: weight tiles [128 x 64] (and, MODE 1, the act tile
 //               [NT x 64]) with the 128-byte swizzle into a STAGES-deep ring.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
-//   warps 2-5   MODE 0 activation gather.  Gather warp g owns every stage whose
-//               sequence number is g mod 4: it issues 16-byte cp.async copies of
-//               the x rows selected by permuted_rows[p] / k straight into the
-//               swizzled B tile (no permuted copy of x exists), waits for them,
-//               then fence.proxy.async and one mbarrier arrival -- the writer-side
-//               proxy fence and barrier the FlashInfer PR #7368 page ("2. Hopper")
-//               requires before an async proxy reads generic-proxy stores.  The
-//               weight TMA of a stage is issued independently of its gather, so
-//               the two overlap (the BF16 ordering of the same section), and four
-//               stages can be in gather at once.
+//   warps 2-7   MODE 0 activation gather, in G = min(6, stages) groups of 6 / G
+//               warps; group g owns every stage whose sequence number is g mod G.
+//               It issues 16-byte cp.async copies of the x rows selected by
+//               permuted_rows[p] / k straight into the swizzled B tile (no permuted
+//               copy of x exists), waits for them, then fence.proxy.async and one
+//               mbarrier arrival per warp -- the writer-side proxy fence and barrier
+//               the FlashInfer PR #7368 page ("2. Hopper") requires before an async
+//               proxy reads generic-proxy stores.  The weight TMA of a stage is issued
+//               independently of its gather, so the two overlap (the BF16 ordering of
+//               the same section).  At most one group per stage keeps every waiter
+//               within one mbarrier phase of its slot.  Idle in MODE 1.
 //   warps 8-15  epilogue, two groups of four: tcgen05.ld of the accumulator
 //               (warp w reads TMEM lanes 32*(w%4) ..), group h owning the token
 //               columns [h*NT/2, (h+1)*NT/2); SwiGLU / bf16 rounding / scatter, or
 //               split-K partials.
-//   warps 6-7   idle.
 //
 // Split-K: when there are too few (tile, feature block) units to fill the GPU
 // (decode), each unit's K range is cut into S slices (S chosen on the device
