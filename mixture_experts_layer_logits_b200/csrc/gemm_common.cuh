@@ -71,8 +71,6 @@ struct Aux {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    int last;
-    int pad;
 };
 
 // TMEM columns an epilogue group reads per tcgen05.ld: 16, or 8 when a group's

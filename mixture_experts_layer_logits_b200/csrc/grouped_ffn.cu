@@ -112,7 +112,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&aux->drain, 1);
         aux->abort = 0;
-        aux->last = 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {

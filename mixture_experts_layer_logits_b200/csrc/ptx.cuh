@@ -181,11 +181,8 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last()
 
 // ---------------------------------------------------------------- cp.async (16 B)
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
-}
-// Same, with an L2 cache policy (from createpolicy) for the source lines.
+// 16-byte global -> shared copy (cp.async.cg: L2 only), with an L2 cache policy
+// (from createpolicy) for the source lines.
 __device__ __forceinline__ void cp_async_16_hint(uint32_t dst_smem, const void* src, uint64_t policy)
 {
     asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst_smem),
@@ -198,24 +195,6 @@ __device__ __forceinline__ void cp_async_wait()
 {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-
-// Bulk (non-tensor) copy shared -> global of `bytes` (multiple of 16, both
-// addresses 16-byte aligned), tracked in this thread's bulk async-group.
-__device__ __forceinline__ void bulk_store(void* dst_global, uint32_t src_smem, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst_global),
-                 "r"(src_smem), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until at most N of this thread's bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read()
-{
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-// Wait until all of this thread's bulk groups have completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Make this thread's completed generic-proxy shared-memory writes visible to
 // async-proxy readers (TMA, tcgen05.mma) ordered after a later synchronisation.
