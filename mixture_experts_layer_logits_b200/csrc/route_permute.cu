@@ -36,14 +36,16 @@ __device__ __forceinline__ bool key_before(float va, int ia, float vb, int ib)
     return va > vb || (va == vb && ia < ib);
 }
 
-// Sorts one (value, index) key per lane across the warp so that lane 0 holds the
-// key that ranks first (larger value, then lower index).  Bitonic network with
+// Sorts one (value, index) key per lane across groups of W lanes (W = 16: each
+// half-warp on its own; W = 32: the warp) so that the group's first lane holds
+// the key that ranks first (larger value, then lower index).  Bitonic network with
 // the "ranks before" relation as the order; keys must be distinct (they are:
 // indices are unique).
+template <int W>
 __device__ __forceinline__ void warp_sort_keys(float& v, int& i, int lane)
 {
 #pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
+    for (int size = 2; size <= W; size <<= 1) {
 #pragma unroll
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             const float ov = __shfl_xor_sync(kFull, v, stride);
@@ -128,9 +130,16 @@ __device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, in
     for (int m = 0; m < V; ++m) mv = fmaxf(mv, v[m]);
     const float tau = __shfl_sync(kFull, warp_sort_desc(mv, lane), k - 1);
 
+    // when E = 32 V every slot holds an expert and the range test can go
+    const bool full = E == 32 * V;
     int c = 0;
+    if (full) {
 #pragma unroll
-    for (int m = 0; m < V; ++m) c += (slot_expert<V, VEC>(m, lane) < E && v[m] >= tau) ? 1 : 0;
+        for (int m = 0; m < V; ++m) c += v[m] >= tau ? 1 : 0;
+    } else {
+#pragma unroll
+        for (int m = 0; m < V; ++m) c += (slot_expert<V, VEC>(m, lane) < E && v[m] >= tau) ? 1 : 0;
+    }
     int incl = c;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -143,10 +152,17 @@ __device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, in
     int my_id = 0;
     if (total <= 32) {
         int pos = incl - c;
+        if (full) {
 #pragma unroll
-        for (int m = 0; m < V; ++m) {
-            const int e = slot_expert<V, VEC>(m, lane);
-            if (e < E && v[m] >= tau) cand[pos++] = make_float2(v[m], __int_as_float(e));
+            for (int m = 0; m < V; ++m)
+                if (v[m] >= tau)
+                    cand[pos++] = make_float2(v[m], __int_as_float(slot_expert<V, VEC>(m, lane)));
+        } else {
+#pragma unroll
+            for (int m = 0; m < V; ++m) {
+                const int e = slot_expert<V, VEC>(m, lane);
+                if (e < E && v[m] >= tau) cand[pos++] = make_float2(v[m], __int_as_float(e));
+            }
         }
         __syncwarp();
         float cv = -INFINITY;
@@ -157,7 +173,12 @@ __device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, in
             ci = __float_as_int(cc.y);
         }
         __syncwarp();  // cand may be rewritten by this warp's next token
-        warp_sort_keys(cv, ci, lane);
+        // usually about k candidates: then lanes 0..15 hold all of them and a
+        // half-warp network (10 stages instead of 15) orders them the same way
+        if (total <= 16)
+            warp_sort_keys<16>(cv, ci, lane);
+        else
+            warp_sort_keys<32>(cv, ci, lane);
         my_l = cv;
         my_id = ci;
     } else {
