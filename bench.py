@@ -404,10 +404,12 @@ def routing_bench(args, w, rank, world, local, dev, pg):
     peaks, peak_kind = load_peaks()
     route_bytes = T * E * 4 + R * 8
     perm_bytes = R * 4 + (E + 1) * 4 + R * 4
-    dominant, dom_ms, dom_bytes = ("route", route_ms, route_bytes) if route_ms >= perm_ms else \
-        ("permute", perm_ms, perm_bytes)
-    roof = roofline_entry(dominant, dict(bytes=dom_bytes, flops=0), dom_ms, peaks, peak_kind,
-                          False, NCU_TRAFFIC.get((w.name, dominant)))
+    # The dominant KERNEL is the routing kernel: the permute stage is two kernels
+    # (per-chunk counts, then the scatter), each shorter than routing in the ncu
+    # launch list (profiles/launches_routing_stress.md), and latency-bound on 1 MB.
+    roof = roofline_entry("route", dict(bytes=route_bytes, flops=0), route_ms, peaks, peak_kind,
+                          False, NCU_TRAFFIC.get((w.name, "route")))
+    roof["permute_ms"] = round(perm_ms, 5)  # count + scatter, for reference
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
