@@ -591,207 +591,6 @@ def main(argv=None):
     if not torch.equal(out_h.to(dev), out):
         raise SystemExit("end-to-end output differs from the device copy")
     e2e_ms = slowest(statistics.mean(a.elapsed_time(b) for a, b in eev))
-
-    peaks, peak_kind = load_peaks()
-    route_bytes = T * E * 4 + R * 8
-    perm_bytes = R * 4 + (E + 1) * 4 + R * 4
-    # The dominant KERNEL is the routing kernel: the permute stage is two kernels
-    # (per-chunk counts, then the scatter), each shorter than routing in the ncu
-    # launch list (profiles/launches_routing_stress.md), and latency-bound on 1 MB.
-    roof = roofline_entry("route", dict(bytes=route_bytes, flops=0), route_ms, peaks, peak_kind,
-                          False, NCU_TRAFFIC.get((w.name, "route")))
-    roof["permute_ms"] = round(perm_ms, 5)  # count + scatter, for reference
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-
-        lg = logits.cpu().numpy()
-        n = 0
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < args.cpu_seconds:
-            rid, _ = oracle.route(lg, k)
-            oracle.permute(rid, E)
-            n += 1
-        dt = time.perf_counter() - t0
-        cpu = {"value": round(n * T / dt, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
-               "kind": "oracle", "sample": f"all {T} tokens (route + permute) x {n} in {dt:.1f} s"}
-    if rank == 0:
-        all_bytes = route_bytes + perm_bytes
-        launches = 1 + (1 if R <= 4096 else 2)
-        line = {
-            "metric": metric_name(w), "value": round(weak_scaling_value(world, T, ms), 2),
-            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": round(ms, 5), "ms_per_step_stats": stats,
-            "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
-            "config": dict(w.as_dict(), parallelism=f"replicas{world}",
-                           l2="flushed before every step (256 MiB write), outside the step events"),
-            "roofline": roof,
-            "stage_ms": {"route": round(route_ms, 5), "permute": round(perm_ms, 5)},
-            "step_GB/s": round(all_bytes / (ms / 1e3) / 1e9, 1),
-            "e2e": {"value": round(world * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
-                    "h2d_bytes_per_step": logits_h.numel() * 4,
-                    "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in outs_h),
-                    "ms_per_step": round(e2e_ms, 5)},
-            "cpu_baseline": cpu,
-            "gpu_launches": launches * (K + KC + W),
-            "gpu_launches_timed_region": launches * K,
-            "clocks": clocks.report(),
-            "wall_s_timed_region": round(t_wall, 4),
-        }
-        print(json.dumps(line), flush=True)
-    if pg:
-        pg.barrier()
-        pg.destroy_process_group()
-
-
-def metric_name(w):
-    return ("MoE layer forward tokens/s at 1 B200 (us/layer in ms_per_step)" if w.has_ffn
-            else "MoE routing (route + permute) tokens/s at 1 B200")
-
-
-# ---------------------------------------------------------------- our arm
-
-def main(argv=None):
-    args = parse_args(argv)
-    rank, world, local = dist_env()
-    if args.impl == "reference":
-        return reference_arm(args, rank, world)
-
-    import numpy as np
-    import torch
-
-    import mixture_experts_layer_logits_b200 as moe
-    from mixture_experts_layer_logits_b200 import build as cuda_build
-    from mixture_experts_layer_logits_b200 import workloads as wl
-
-    if rank == 0:
-        cuda_build.build()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-        pg = dist
-        dist.barrier()
-    moe.load_library()
-
-    w = get_workload(args.workload)
-    if not w.has_ffn:
-        return routing_bench(args, w, rank, world, local, dev, pg)
-    T, E, k, H, I = w.T, w.E, w.k, w.H, w.I
-    R = T * k
-    # this rank's tokens; weights are the same on every rank
-    logits = wl.make_logits(w, seed=rank_seed(args.seed, rank), device=dev)
-    x = wl.make_x(w, seed=rank_seed(args.seed, rank), device=dev)
-    w13, w2 = wl.make_weights(w, seed=args.seed, device=dev)
-    ws = moe.workspace(T, E, k, H, I, device=dev)
-    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
-    wts = torch.empty(T, k, dtype=torch.float32, device=dev)
-    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    rows = torch.empty(R, dtype=torch.int32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def fwd():
-        moe.moe_forward(x, logits, w13, w2, k, ws=ws, out=out, topk_ids=ids, topk_weights=wts,
-                        expert_offsets=off, permuted_rows=rows)
-
-    def barrier():
-        torch.cuda.synchronize(dev)
-        if pg:
-            pg.barrier()
-
-    def slowest(v):
-        return max_over_ranks(v, pg, dev)
-
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        fwd()
-    barrier()
-    if moe.moe_device_status(ws) != moe.MOE_OK:
-        raise SystemExit("device error during warm-up")
-    n_touched = int((off[1:] - off[:-1] > 0).sum().item())
-
-    # ---- pass A: the timed steps
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
-    barrier()
-    with ClockSampler(local) as clocks:
-        t_wall = time.perf_counter()
-        torch.cuda.nvtx.range_push("timed")  # lets a profiler select the timed steps
-        for i in range(K):
-            flush.zero_()
-            ev[i][0].record(stream)
-            fwd()
-            ev[i][1].record(stream)
-        torch.cuda.nvtx.range_pop()
-        barrier()
-        t_wall = time.perf_counter() - t_wall
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = slowest(statistics.mean(step_ms))
-    stats = step_stats(step_ms, slowest)
-    if moe.moe_device_status(ws) != moe.MOE_OK:
-        raise SystemExit("device error during the timed steps")
-
-    # ---- pass B: stage durations through moe_forward_timed
-    KB = min(K, 200)
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(KB)]
-    for evs in sev:  # materialise the events (torch creates them on first record)
-        for e in evs:
-            e.record(stream)
-    barrier()
-    for i in range(KB):
-        flush.zero_()
-        moe.moe_forward_timed(x, logits, w13, w2, k, sev[i], ws=ws, out=out, topk_ids=ids,
-                              topk_weights=wts, expert_offsets=off, permuted_rows=rows)
-    barrier()
-    fused = moe.moe_forward_fused(T, E, k, H, I)
-    if fused:  # events 2..4 all follow the one FFN + combine launch
-        spans = {"route_permute": (0, 1), "fused_ffn": (1, 4)}
-    else:
-        spans = {"route_permute": (0, 1), "w13": (1, 2), "w2": (2, 3), "combine": (3, 4)}
-    stage_ms = {n: statistics.mean(sev[i][a].elapsed_time(sev[i][b]) for i in range(KB))
-                for n, (a, b) in spans.items()}
-    stage_ms = {n: slowest(v) for n, v in stage_ms.items()}
-
-    # ---- pass C: end to end from pinned host memory.  The step's inputs (x, then
-    # logits at a 256-byte aligned offset) sit in one pinned host buffer and cross
-    # in one copy to one device buffer whose views the forward reads; out comes
-    # back in one copy.
-    KC = min(K, 200)
-    xb = x.numel() * x.element_size()
-    lo = (xb + 255) // 256 * 256
-    lb = logits.numel() * logits.element_size()
-    in_h = torch.empty(lo + lb, dtype=torch.uint8).pin_memory()
-    in_h[:xb].copy_(x.cpu().view(-1).view(torch.uint8))
-    in_h[lo:].copy_(logits.cpu().view(-1).view(torch.uint8))
-    in_d = torch.empty(lo + lb, dtype=torch.uint8, device=dev)
-    x_e = in_d[:xb].view(torch.bfloat16).view(T, H)
-    logits_e = in_d[lo:].view(torch.float32).view(T, E)
-    out_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(KC)]
-    barrier()
-    for i in range(KC):
-        flush.zero_()
-        eev[i][0].record(stream)
-        in_d.copy_(in_h, non_blocking=True)
-        moe.moe_forward(x_e, logits_e, w13, w2, k, ws=ws, out=out, topk_ids=ids,
-                        topk_weights=wts, expert_offsets=off, permuted_rows=rows)
-        out_h.copy_(out, non_blocking=True)
-        eev[i][1].record(stream)
-    barrier()
-    if not torch.equal(out_h.to(dev), out):
-        raise SystemExit("end-to-end output differs from the device copy")
-    e2e_ms = slowest(statistics.mean(a.elapsed_time(b) for a, b in eev))
     h2d = x_h.numel() * x_h.element_size() + logits_h.numel() * logits_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 
