@@ -183,7 +183,10 @@ moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, cons
             gemm::make_tmap(&pf, w13_prefetch, (uint64_t)s.E * 2 * s.I, (uint64_t)s.H, gemm::kBM) ==
                 cudaSuccess) {
             pf_map = &pf;
-            aux.pf_units = device_sms();  // the fused grid: each CTA's first w13 unit
+            // each fused CTA's first w13 unit, as far as there can be w13 units:
+            // at most min(E, T*k) tiles (one per touched expert), I/128 units each
+            const long max_units13 = (long)(s.E < R ? s.E : R) * (s.I / gemm::kBM);
+            aux.pf_units = (int)(max_units13 < device_sms() ? max_units13 : device_sms());
             aux.pf_fb13 = s.I / gemm::kBM;
             aux.pf_I = s.I;
             // 16 K tiles (2 x 128 x 1024 weights per CTA) cover the routing and
