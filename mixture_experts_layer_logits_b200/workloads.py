@@ -132,6 +132,35 @@ def make_weights(w: Workload, seed: int = 0, device="cpu"):
     return w13, w2
 
 
+E4M3_MAX = 448.0  # largest finite E4M3 (E4M3FN) value
+
+
+def quantize_e4m3_rows(t: torch.Tensor):
+    """Symmetric per-row E4M3 quantisation of a [..., rows, cols] weight tensor:
+    scale = max|row| / 448 (1 for an all-zero row), codes = the E4M3 value nearest
+    to w / scale.  Returns (codes uint8 [..., rows, cols], scales float32
+    [..., rows]).  Input preparation only: the layer reads codes and scales."""
+    tf = t.float()
+    amax = tf.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    q = (tf / scale.unsqueeze(-1)).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8), scale
+
+
+def make_weights_w8(w: Workload, seed: int = 0, device="cpu"):
+    """FP8 copies of make_weights' draws, quantised one expert at a time:
+    (q13 uint8 [E,2I,H], s13 f32 [E,2I], q2 uint8 [E,H,I], s2 f32 [E,H])."""
+    q13 = torch.empty(w.E, 2 * w.I, w.H, dtype=torch.uint8, device=device)
+    s13 = torch.empty(w.E, 2 * w.I, dtype=torch.float32, device=device)
+    q2 = torch.empty(w.E, w.H, w.I, dtype=torch.uint8, device=device)
+    s2 = torch.empty(w.E, w.H, dtype=torch.float32, device=device)
+    for e in range(w.E):
+        a, b = make_expert_weights(w, e, seed, device)
+        q13[e], s13[e] = quantize_e4m3_rows(a)
+        q2[e], s2[e] = quantize_e4m3_rows(b)
+    return q13, s13, q2, s2
+
+
 def make_inputs(w: Workload, seed: int = 0, device="cpu", weights: bool = True) -> dict:
     d = dict(logits=make_logits(w, seed, device))
     if w.has_ffn:

@@ -7,7 +7,8 @@ library and its binding) never does, and shares no code with it.
 Thin ctypes wrapper over ``moe_oracle.c`` (compiled by ``oracle/build.py`` into
 ``oracle/libmoe_oracle.so``).  Inputs are numpy arrays on the host: logits
 float32 [T,E]; x bf16 bits as uint16 [T,H]; w13 uint16 [E,2I,H]; w2 uint16
-[E,H,I].  What each function computes, and the passages it follows, is stated in
+[E,H,I]; FP8 weights as uint8 E4M3 codes (q13 [E,2I,H], q2 [E,H,I]) with
+float32 per-row scales (s13 [E,2I], s2 [E,H]).  What each function computes, and the passages it follows, is stated in
 ``moe_oracle.c``.
 """
 from __future__ import annotations
@@ -25,6 +26,7 @@ _i32p = ctypes.POINTER(ctypes.c_int32)
 _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 
 
 def _load():
@@ -46,9 +48,17 @@ def _load():
     lib.oracle_forward_tokens.argtypes = [_u16p, _f32p, ctypes.POINTER(_u16p),
                                           ctypes.POINTER(_u16p), i, i, i, i, i, i, i, _i32p,
                                           _f64p]
+    lib.oracle_e4m3_to_double.argtypes = [_u8p, ctypes.c_long, _f64p]
+    lib.oracle_forward_w8.argtypes = [_u16p, _f32p, _u8p, _f32p, _u8p, _f32p, i, i, i, i, i,
+                                      _f64p, _i32p, _f32p, _i32p, _i32p]
+    lib.oracle_forward_tokens_w8.argtypes = [_u16p, _f32p, ctypes.POINTER(_u8p),
+                                             ctypes.POINTER(_f32p), ctypes.POINTER(_u8p),
+                                             ctypes.POINTER(_f32p), i, i, i, i, i, i, _i32p,
+                                             _f64p]
     lib.oracle_num_threads.argtypes = []
     for fn in (lib.oracle_num_threads, lib.oracle_route, lib.oracle_permute, lib.oracle_ffn, lib.oracle_combine,
-               lib.oracle_forward, lib.oracle_forward_tokens):
+               lib.oracle_forward, lib.oracle_forward_tokens, lib.oracle_e4m3_to_double,
+               lib.oracle_forward_w8, lib.oracle_forward_tokens_w8):
         fn.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -180,5 +190,72 @@ def forward_tokens(x, logits, w13_experts, w2_experts, k, tokens, I, round_inter
     if rc == -3:
         raise ValueError("a listed token selects an expert whose weights were not given")
     _check(rc, "forward_tokens")
+    del keep
+    return out
+
+
+def e4m3_to_float64(q):
+    """E4M3 (E4M3FN) codes (uint8) -> float64 values, NaN for 0x7F / 0xFF."""
+    q = _c(q, np.uint8)
+    out = np.empty(q.shape, np.float64)
+    _check(_load().oracle_e4m3_to_double(_p(q, _u8p), q.size, _p(out, _f64p)), "e4m3_to_double")
+    return out
+
+
+def forward_w8(x, logits, q13, s13, q2, s2, k):
+    """Whole layer with FP8 weights: weight = e4m3(q) * per-row scale.  Returns the
+    same dict as forward()."""
+    x = _c(x, np.uint16)
+    logits = _c(logits, np.float32)
+    q13 = _c(q13, np.uint8)
+    q2 = _c(q2, np.uint8)
+    s13 = _c(s13, np.float32)
+    s2 = _c(s2, np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    I = q13.shape[1] // 2
+    if q13.shape != (E, 2 * I, H) or q2.shape != (E, H, I) or s13.shape != (E, 2 * I) \
+            or s2.shape != (E, H):
+        raise ValueError("FP8 weight or scale shapes do not match")
+    out = np.empty((T, H), np.float64)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    off = np.empty(E + 1, np.int32)
+    rows = np.empty(T * k, np.int32)
+    _check(_load().oracle_forward_w8(_p(x, _u16p), _p(logits, _f32p), _p(q13, _u8p),
+                                     _p(s13, _f32p), _p(q2, _u8p), _p(s2, _f32p), T, E, k, H, I,
+                                     _p(out, _f64p), _p(ids, _i32p), _p(w, _f32p),
+                                     _p(off, _i32p), _p(rows, _i32p)), "forward_w8")
+    return dict(out=out, topk_ids=ids, topk_weights=w, expert_offsets=off, permuted_rows=rows)
+
+
+def forward_tokens_w8(x, logits, experts, k, tokens, I):
+    """Layer output of the listed tokens only, FP8 weights.  ``experts`` is a
+    length-E sequence whose entry e is (q13 [2I,H] uint8, s13 [2I] f32,
+    q2 [H,I] uint8, s2 [H] f32), or None for an expert the tokens do not select.
+    Returns float64 [len(tokens), H]."""
+    x = _c(x, np.uint16)
+    logits = _c(logits, np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    keep = []
+    q13p, s13p, q2p, s2p = (_u8p * E)(), (_f32p * E)(), (_u8p * E)(), (_f32p * E)()
+    for e in range(E):
+        if experts[e] is None:
+            continue
+        a, sa, b, sb = (_c(experts[e][0], np.uint8), _c(experts[e][1], np.float32),
+                        _c(experts[e][2], np.uint8), _c(experts[e][3], np.float32))
+        if a.shape != (2 * I, H) or sa.shape != (2 * I,) or b.shape != (H, I) or sb.shape != (H,):
+            raise ValueError(f"expert {e}: bad FP8 weight or scale shapes")
+        keep += [a, sa, b, sb]
+        q13p[e], s13p[e], q2p[e], s2p[e] = _p(a, _u8p), _p(sa, _f32p), _p(b, _u8p), _p(sb, _f32p)
+    toks = np.ascontiguousarray(np.asarray(tokens, np.int32))
+    out = np.empty((len(toks), H), np.float64)
+    rc = _load().oracle_forward_tokens_w8(_p(x, _u16p), _p(logits, _f32p), q13p, s13p, q2p, s2p,
+                                          T, E, k, H, I, len(toks), _p(toks, _i32p),
+                                          _p(out, _f64p))
+    if rc == -3:
+        raise ValueError("a listed token selects an expert whose weights were not given")
+    _check(rc, "forward_tokens_w8")
     del keep
     return out

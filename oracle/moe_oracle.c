@@ -36,9 +36,18 @@
  * on an invalid argument (null pointer, non-positive size, k > E, an expert id
  * out of range); outputs are then left untouched.
  *
+ * FP8 weights (the *_w8 entry points): w13 and w2 arrive as E4M3 codes (the
+ * OCP "E4M3FN" format: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * subnormals, no infinities, 0x7F / 0xFF are NaN) with one fp32 scale per weight
+ * row (per output feature): the weight is e4m3(q) * scale, exact in double.  The
+ * layer is otherwise the same four steps.
+ *
  * Pinned by tests/test_oracle_pins.py (closed forms of a hand-worked example,
  * rank-count brute force, invariants, reduction to library softmax / a plain
- * SwiGLU MLP, and a dense all-experts masked loop).
+ * SwiGLU MLP, and a dense all-experts masked loop; for the FP8 weights, the
+ * E4M3 decoder against a library conversion of every code, bit equality with
+ * the bf16 layer when the dequantised weights are bf16 values, and a dense
+ * dequantise-then-multiply check).
  */
 #include <math.h>
 #include <omp.h>
@@ -50,6 +59,25 @@
 int oracle_num_threads(void) { return omp_get_max_threads(); }
 
 /* ---- exact upcasts ------------------------------------------------------ */
+
+/* E4M3 (E4M3FN) code -> double, from the format's definition: exponent field
+ * 0 encodes subnormals m * 2^-9; otherwise (1 + m/8) * 2^(e - 7); the all-ones
+ * code (exponent 15, mantissa 7) of either sign is NaN; there is no infinity. */
+static double e4m3_to_double(uint8_t q)
+{
+    const int sign = q >> 7, e = (q >> 3) & 15, m = q & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* Decodes n E4M3 codes (exported for the pins). */
+int oracle_e4m3_to_double(const uint8_t* q, long n, double* out)
+{
+    if (!q || !out || n < 0) return -1;
+    for (long i = 0; i < n; ++i) out[i] = e4m3_to_double(q[i]);
+    return 0;
+}
 
 /* bf16 bit pattern -> double (exact: bf16 is the top half of an fp32). */
 static double bf16_to_double(uint16_t b)
@@ -305,6 +333,132 @@ int oracle_forward_tokens(const uint16_t* x, const float* logits,
                     if (!w13_e[e] || !w2_e[e]) { missing = 1; break; }
                     expert_ffn_row(x + (size_t)t * H, w13_e[e], w2_e[e], H, I,
                                    round_intermediates, act, yk + (size_t)j * H);
+                }
+                if (missing) {
+#pragma omp atomic write
+                    bad = -3;
+                    continue;
+                }
+                for (int h = 0; h < H; ++h) {
+                    double acc = 0.0;
+                    for (int j = 0; j < k; ++j) acc += (double)w[j] * yk[(size_t)j * H + h];
+                    out_sel[(size_t)s * H + h] = acc;
+                }
+            }
+        }
+        free(scratch);
+        free(act);
+        free(yk);
+        free(ids);
+        free(w);
+    }
+    return bad;
+}
+
+/* ---- FP8 weights ------------------------------------------------------------ */
+
+/* As expert_ffn_row with w13_e = [2I, H] E4M3 codes and s13_e = [2I] row scales,
+ * w2_e = [H, I] codes and s2_e = [H] row scales: weight (r, c) = e4m3(q) * s[r]. */
+static void expert_ffn_row_w8(const uint16_t* x_row, const uint8_t* q13_e, const float* s13_e,
+                              const uint8_t* q2_e, const float* s2_e, int H, int I, double* act,
+                              double* y_row)
+{
+    for (int c = 0; c < I; ++c) {
+        const uint8_t* qg = q13_e + (size_t)c * H;
+        const uint8_t* qu = q13_e + (size_t)(I + c) * H;
+        const double sg = s13_e[c], su = s13_e[I + c];
+        double gate = 0.0, up = 0.0;
+        for (int i = 0; i < H; ++i) {
+            const double xi = bf16_to_double(x_row[i]);
+            gate += xi * (e4m3_to_double(qg[i]) * sg);
+            up += xi * (e4m3_to_double(qu[i]) * su);
+        }
+        act[c] = gate / (1.0 + exp(-gate)) * up;
+    }
+    for (int o = 0; o < H; ++o) {
+        const uint8_t* q = q2_e + (size_t)o * I;
+        const double so = s2_e[o];
+        double acc = 0.0;
+        for (int c = 0; c < I; ++c) acc += act[c] * (e4m3_to_double(q[c]) * so);
+        y_row[o] = acc;
+    }
+}
+
+/* The whole layer with FP8 weights: q13 [E, 2I, H] codes + s13 [E, 2I] scales,
+ * q2 [E, H, I] codes + s2 [E, H] scales; outputs as oracle_forward. */
+int oracle_forward_w8(const uint16_t* x, const float* logits, const uint8_t* q13, const float* s13,
+                      const uint8_t* q2, const float* s2, int T, int E, int k, int H, int I,
+                      double* out, int32_t* topk_ids, float* topk_weights,
+                      int32_t* expert_offsets, int32_t* permuted_rows)
+{
+    if (!x || !q13 || !s13 || !q2 || !s2 || !out || H < 1 || I < 1) return -1;
+    int rc = oracle_route(logits, T, E, k, topk_ids, topk_weights);
+    if (rc) return rc;
+    rc = oracle_permute(topk_ids, T, k, E, expert_offsets, permuted_rows);
+    if (rc) return rc;
+    const long R = (long)T * k;
+    double* y = (double*)malloc(sizeof(double) * (size_t)R * H);
+    if (!y) return -2;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* act = (double*)malloc(sizeof(double) * (size_t)I);
+        if (!act) {
+#pragma omp atomic write
+            bad = -2;
+        } else {
+            for (int e = 0; e < E; ++e) {
+#pragma omp for schedule(dynamic, 1)
+                for (long p = expert_offsets[e]; p < expert_offsets[e + 1]; ++p) {
+                    const long r = permuted_rows[p];
+                    expert_ffn_row_w8(x + (size_t)(r / k) * H, q13 + (size_t)e * 2 * I * H,
+                                      s13 + (size_t)e * 2 * I, q2 + (size_t)e * H * I,
+                                      s2 + (size_t)e * H, H, I, act, y + (size_t)r * H);
+                }
+            }
+            free(act);
+        }
+    }
+    if (!bad) bad = oracle_combine(y, topk_weights, T, k, H, out);
+    free(y);
+    return bad;
+}
+
+/* oracle_forward_tokens with FP8 weights: per-expert pointer tables of codes
+ * (q13_e[e] -> [2I, H], q2_e[e] -> [H, I]) and scales (s13_e[e] -> [2I],
+ * s2_e[e] -> [H]); a selected expert with a NULL entry is an error (-3). */
+int oracle_forward_tokens_w8(const uint16_t* x, const float* logits,
+                             const uint8_t* const* q13_e, const float* const* s13_e,
+                             const uint8_t* const* q2_e, const float* const* s2_e, int T, int E,
+                             int k, int H, int I, int n_sel, const int32_t* tokens,
+                             double* out_sel)
+{
+    if (!x || !logits || !q13_e || !s13_e || !q2_e || !s2_e || !tokens || !out_sel) return -1;
+    if (T < 1 || E < 1 || k < 1 || k > E || H < 1 || I < 1 || n_sel < 0) return -1;
+    for (int s = 0; s < n_sel; ++s)
+        if (tokens[s] < 0 || tokens[s] >= T) return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        route_key* scratch = (route_key*)malloc(sizeof(route_key) * (size_t)E);
+        double* act = (double*)malloc(sizeof(double) * (size_t)I);
+        double* yk = (double*)malloc(sizeof(double) * (size_t)k * H);
+        int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+        float* w = (float*)malloc(sizeof(float) * (size_t)k);
+        if (!scratch || !act || !yk || !ids || !w) {
+#pragma omp atomic write
+            bad = -2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int s = 0; s < n_sel; ++s) {
+                const int t = tokens[s];
+                route_one_token(logits + (size_t)t * E, E, k, scratch, ids, w);
+                int missing = 0;
+                for (int j = 0; j < k; ++j) {
+                    const int e = ids[j];
+                    if (!q13_e[e] || !s13_e[e] || !q2_e[e] || !s2_e[e]) { missing = 1; break; }
+                    expert_ffn_row_w8(x + (size_t)t * H, q13_e[e], s13_e[e], q2_e[e], s2_e[e], H,
+                                      I, act, yk + (size_t)j * H);
                 }
                 if (missing) {
 #pragma omp atomic write

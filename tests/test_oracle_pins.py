@@ -6,6 +6,9 @@
 * special cases that reduce to library routines (torch.softmax for k = E,
   torch.nn.functional.silu + matmul for a one-expert layer);
 * a dense loop over all experts masked by the routing weights (no permutation);
+* FP8 weights: the E4M3 decoder against the library conversion of all 256 codes,
+  bit equality with the bf16 layer on bf16-exact dequantised weights, and a
+  dense dequantise-then-multiply loop;
 * planted mistakes: a mutated copy of the oracle must fail these pins.
 """
 import json
@@ -307,6 +310,104 @@ def test_workload_inputs_deterministic_and_shaped():
     assert abs(float(torch.exp(z.double() / 2).sum()) - 1.0) < 1e-6
 
 
+# ---------------------------------------------------------------- FP8 (E4M3) weights
+
+def _rand_w8_layer(rng, T, E, k, H, I, pow2_scales):
+    """Random E4M3 codes (no NaN codes) and positive per-row scales."""
+    logits, x, _, _ = _rand_layer(rng, T, E, k, H, I)
+
+    def codes(shape):
+        q = rng.integers(0, 256, shape, dtype=np.uint8)
+        q[(q & 0x7F) == 0x7F] = 0x7E  # NaN codes -> 448 of the same sign
+        return q
+
+    def scales(shape):
+        if pow2_scales:
+            return (2.0 ** rng.integers(-9, -3, shape)).astype(np.float32)
+        return rng.uniform(1e-3, 1e-2, shape).astype(np.float32)
+
+    return (logits, x, codes((E, 2 * I, H)), scales((E, 2 * I)), codes((E, H, I)),
+            scales((E, H)))
+
+
+def _e4m3_library(q):
+    return torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def test_e4m3_decoder_is_the_library_conversion():
+    """Every one of the 256 codes decodes to PyTorch's float8_e4m3fn value."""
+    q = np.arange(256, dtype=np.uint8)
+    got, want = oracle.e4m3_to_float64(q), _e4m3_library(q)
+    nan = np.isnan(want)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    assert np.isnan(got[nan]).all()
+    np.testing.assert_array_equal(got[~nan], want[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x80] == 0.0
+
+
+@pytest.mark.parametrize("T,E,k,H,I", [(5, 6, 3, 8, 4), (9, 4, 4, 16, 8), (3, 1, 1, 8, 8)])
+def test_w8_layer_equals_bf16_layer_on_bf16_exact_weights(T, E, k, H, I):
+    """With power-of-two scales every dequantised weight is a bf16 value, and the
+    FP8 layer must equal the bf16 layer on those weights bit for bit."""
+    rng = np.random.default_rng(T * 7 + E)
+    logits, x, q13, s13, q2, s2 = _rand_w8_layer(rng, T, E, k, H, I, pow2_scales=True)
+    w13 = _e4m3_library(q13) * s13[..., None]
+    w2 = _e4m3_library(q2) * s2[..., None]
+    to_bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    b13, b2 = to_bits(w13), to_bits(w2)
+    np.testing.assert_array_equal(_bits_to_f64(b13), w13)  # the premise: exact in bf16
+    ref = oracle.forward(x, logits, b13, b2, k)
+    got = oracle.forward_w8(x, logits, q13, s13, q2, s2, k)
+    for key in ("topk_ids", "topk_weights", "expert_offsets", "permuted_rows", "out"):
+        np.testing.assert_array_equal(got[key], ref[key])
+
+
+@pytest.mark.parametrize("T,E,k,H,I", [(5, 6, 3, 8, 4), (12, 10, 2, 32, 24)])
+def test_w8_dense_dequantised_loop(T, E, k, H, I):
+    """Arbitrary scales: every expert on every token with weights dequantised by
+    the library (code value * row scale), masked by the routing weights."""
+    rng = np.random.default_rng(T * 13 + E)
+    logits, x, q13, s13, q2, s2 = _rand_w8_layer(rng, T, E, k, H, I, pow2_scales=False)
+    res = oracle.forward_w8(x, logits, q13, s13, q2, s2, k)
+    ids, w = res["topk_ids"], res["topk_weights"]
+    X = _bits_to_f64(x)
+    W13 = _e4m3_library(q13) * s13.astype(np.float64)[..., None]
+    W2 = _e4m3_library(q2) * s2.astype(np.float64)[..., None]
+    dense = np.zeros((T, H))
+    for t in range(T):
+        for e in range(E):
+            hit = np.nonzero(ids[t] == e)[0]
+            m = float(w[t, hit[0]]) if len(hit) else 0.0
+            h = W13[e] @ X[t]
+            g, u = h[:I], h[I:]
+            dense[t] += m * (W2[e] @ (g / (1.0 + np.exp(-g)) * u))
+    np.testing.assert_allclose(res["out"], dense, rtol=1e-12, atol=1e-13)
+
+
+def test_w8_forward_tokens_matches_forward_w8():
+    rng = np.random.default_rng(17)
+    T, E, k, H, I = 11, 7, 3, 16, 8
+    logits, x, q13, s13, q2, s2 = _rand_w8_layer(rng, T, E, k, H, I, pow2_scales=False)
+    full = oracle.forward_w8(x, logits, q13, s13, q2, s2, k)["out"]
+    toks = [0, 4, 10]
+    experts = [(q13[e], s13[e], q2[e], s2[e]) for e in range(E)]
+    sel = oracle.forward_tokens_w8(x, logits, experts, k, toks, I)
+    np.testing.assert_array_equal(sel, full[toks])
+
+
+def test_workload_w8_quantisation_reconstructs_weights():
+    w = wl.custom("q", 4, 3, 2, 256, 128)
+    q13, s13, q2, s2 = wl.make_weights_w8(w)
+    w13, w2 = wl.make_weights(w)
+    for q, sc, ref in ((q13, s13, w13), (q2, s2, w2)):
+        deq = _e4m3_library(q.numpy()) * sc.double().numpy()[..., None]
+        r = ref.double().numpy()
+        # E4M3 keeps 3 mantissa bits: round-to-nearest error <= 2^-4 relative, and
+        # every row's largest magnitude maps to 448 exactly
+        np.testing.assert_array_less(np.abs(deq - r), 2.0 ** -4 * np.abs(r) + 2.0 ** -9 * sc.double().numpy()[..., None] + 1e-12)
+        np.testing.assert_allclose(np.abs(deq).max(axis=-1), np.abs(r).max(axis=-1), rtol=1e-6)
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 MUTATIONS = [
@@ -328,6 +429,12 @@ MUTATIONS = [
     ("combine drops the last choice",
      "for (int j = 0; j < k; ++j)\n                acc += (double)topk_weights",
      "for (int j = 0; j + 1 < k; ++j)\n                acc += (double)topk_weights"),
+    ("E4M3 exponent bias 8",
+     "ldexp(1.0 + m / 8.0, e - 7)",
+     "ldexp(1.0 + m / 8.0, e - 8)"),
+    ("FP8 gate and up scales swapped",
+     "const double sg = s13_e[c], su = s13_e[I + c];",
+     "const double sg = s13_e[I + c], su = s13_e[c];"),
 ]
 
 
@@ -350,7 +457,9 @@ def test_planted_mistake_is_caught(name, old, new, monkeypatch, tmp_path):
         for check in (test_hand_example_oracle,
                       lambda: test_route_rank_count_brute_force(40, 8, 2),
                       lambda: test_permute_brute_force_and_invariants(33, 5, 3),
-                      lambda: test_dense_masked_all_experts_loop(5, 6, 3, 8, 4)):
+                      lambda: test_dense_masked_all_experts_loop(5, 6, 3, 8, 4),
+                      test_e4m3_decoder_is_the_library_conversion,
+                      lambda: test_w8_dense_dequantised_loop(5, 6, 3, 8, 4)):
             try:
                 check()
             except AssertionError:
