@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the MoE layer forward on B200 (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--weights bf16|e4m3]
                     [--impl ours|reference]
 
 A step is one whole layer forward (route -> permute -> w13/SwiGLU -> w2 ->
@@ -63,6 +63,9 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="decode",
                    help="a named workload, or custom:T=..,E=..,k=..,H=..,I=..[,zipf=..]")
+    p.add_argument("--weights", choices=["bf16", "e4m3"], default="bf16",
+                   help="expert weight format: bf16, or E4M3 codes with per-row fp32 scales "
+                        "(moe_forward_w8; T <= 64 shapes)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -119,21 +122,27 @@ def load_peaks():
 
 # ---------------------------------------------------------------- stage work model
 
-def stage_work(w, n_touched):
+def stage_work(w, n_touched, weights="bf16"):
     """Algorithmic bytes and FLOPs per launch of each stage (not counting padding
-    or re-reads).  n_touched = experts with at least one routed row."""
+    or re-reads).  n_touched = experts with at least one routed row.  E4M3
+    weights are one byte each plus one fp32 scale per weight row."""
     T, E, k, H, I = w.T, w.E, w.k, w.H, w.I
     R = T * k
+    wb = 1 if weights == "e4m3" else 2
+    s13 = 2 * I * 4 if weights == "e4m3" else 0  # row scales per expert
+    s2 = H * 4 if weights == "e4m3" else 0
     return {
         "route_permute": dict(bytes=T * E * 4 + R * (4 + 4) + R * 4 + (E + 1) * 4, flops=0),
-        "w13": dict(bytes=n_touched * 2 * I * H * 2 + T * H * 2 + R * I * 2,
+        "w13": dict(bytes=n_touched * (2 * I * H * wb + s13) + T * H * 2 + R * I * 2,
                     flops=2 * R * 2 * I * H),
-        "w2": dict(bytes=n_touched * H * I * 2 + R * I * 2 + R * H * 2, flops=2 * R * H * I),
+        "w2": dict(bytes=n_touched * (H * I * wb + s2) + R * I * 2 + R * H * 2,
+                   flops=2 * R * H * I),
         "combine": dict(bytes=R * H * 2 + R * 4 + T * H * 2, flops=0),
         # w13 + w2 + combine as one launch: act and y never need to reach HBM, so
         # the algorithmic bytes are the touched weights, x, the routing weights and
         # permuted rows, and out
-        "fused_ffn": dict(bytes=n_touched * 3 * I * H * 2 + T * H * 2 + R * 8 + T * H * 2,
+        "fused_ffn": dict(bytes=n_touched * (3 * I * H * wb + s13 + s2) + T * H * 2 + R * 8 +
+                          T * H * 2,
                           flops=2 * R * 2 * I * H + 2 * R * H * I),
     }
 
@@ -224,13 +233,16 @@ class ClockSampler:
 # ---------------------------------------------------------------- CPU oracle timing
 
 def oracle_sample(w, d_host, seconds):
-    """Time the fp64 oracle on a bounded sample of the workload; returns tokens/s info."""
+    """Time the fp64 oracle on a bounded sample of the workload; returns tokens/s info.
+    d_host = (x, logits, w13, w2) with bf16 weights, or (x, logits, (q13, s13),
+    (q2, s2)) with E4M3 codes and row scales."""
     import numpy as np
 
     import oracle
 
     T, k, H, I = w.T, w.k, w.H, w.I
     x, logits, w13, w2 = d_host
+    e4m3 = isinstance(w13, tuple)
     per_token_macs = k * 3 * H * I
     full_layer = T * per_token_macs <= 2e9
     done_tokens = 0
@@ -238,7 +250,10 @@ def oracle_sample(w, d_host, seconds):
     t0 = time.perf_counter()
     if full_layer:
         while True:
-            oracle.forward(x, logits, w13, w2, k)
+            if e4m3:
+                oracle.forward_w8(x, logits, w13[0], w13[1], w2[0], w2[1], k)
+            else:
+                oracle.forward(x, logits, w13, w2, k)
             done_tokens += T
             calls += 1
             if time.perf_counter() - t0 >= seconds:
@@ -249,10 +264,17 @@ def oracle_sample(w, d_host, seconds):
         ids, _ = oracle.route(logits, k)
         tok = list(range(n))
         used = set(ids[tok].reshape(-1).tolist())
-        w13s = [w13[e] if e in used else None for e in range(w.E)]
-        w2s = [w2[e] if e in used else None for e in range(w.E)]
+        if e4m3:
+            experts = [(w13[0][e], w13[1][e], w2[0][e], w2[1][e]) if e in used else None
+                       for e in range(w.E)]
+        else:
+            w13s = [w13[e] if e in used else None for e in range(w.E)]
+            w2s = [w2[e] if e in used else None for e in range(w.E)]
         while True:
-            oracle.forward_tokens(x, logits, w13s, w2s, k, tok, I)
+            if e4m3:
+                oracle.forward_tokens_w8(x, logits, experts, k, tok, I)
+            else:
+                oracle.forward_tokens(x, logits, w13s, w2s, k, tok, I)
             done_tokens += n
             calls += 1
             if time.perf_counter() - t0 >= seconds:
@@ -285,13 +307,23 @@ def reference_arm(args, rank, world):
         used = sorted(set(ids[tok].reshape(-1).tolist()))
         w13s = [None] * w.E
         w2s = [None] * w.E
+        experts = [None] * w.E
         for e in used:
             a, b = wl.make_expert_weights(w, e, seed=args.seed, device="cpu")
-            w13s[e], w2s[e] = wl.bf16_bits(a), wl.bf16_bits(b)
+            if args.weights == "e4m3":
+                (qa, sa), (qb, sb) = wl.quantize_e4m3_rows(a), wl.quantize_e4m3_rows(b)
+                experts[e] = (qa.numpy(), sa.numpy(), qb.numpy(), sb.numpy())
+            else:
+                w13s[e], w2s[e] = wl.bf16_bits(a), wl.bf16_bits(b)
 
         def step():
-            oracle.forward_tokens(x, logits, w13s, w2s, w.k, tok, w.I)
+            if args.weights == "e4m3":
+                oracle.forward_tokens_w8(x, logits, experts, w.k, tok, w.I)
+            else:
+                oracle.forward_tokens(x, logits, w13s, w2s, w.k, tok, w.I)
             return n
+        if args.weights == "e4m3":
+            cfg["weights"] = "e4m3 + fp32 row scales"
         sample = f"{n} of {w.T} tokens per step"
         metric_unit = "tokens/s"
     else:
@@ -434,6 +466,8 @@ def routing_bench(args, w, rank, world, local, dev, pg):
             "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
             "config": dict(w.as_dict(), parallelism=f"replicas{world}",
+                           weights=("e4m3 codes + fp32 row scales (moe_forward_w8)" if e4m3
+                                    else "bf16"),
                            l2="flushed before every step (256 MiB write), outside the step events"),
             "roofline": roof,
             "stage_ms": {"route": round(route_ms, 5), "permute": round(perm_ms, 5)},
@@ -498,7 +532,13 @@ def main(argv=None):
     # this rank's tokens; weights are the same on every rank
     logits = wl.make_logits(w, seed=rank_seed(args.seed, rank), device=dev)
     x = wl.make_x(w, seed=rank_seed(args.seed, rank), device=dev)
-    w13, w2 = wl.make_weights(w, seed=args.seed, device=dev)
+    e4m3 = args.weights == "e4m3"
+    if e4m3:
+        if not moe.moe_forward_w8_supported(T, E, k, H, I):
+            raise SystemExit(f"--weights e4m3: moe_forward_w8 does not take {w.name}")
+        q13, s13, q2, s2 = wl.make_weights_w8(w, seed=args.seed, device=dev)
+    else:
+        w13, w2 = wl.make_weights(w, seed=args.seed, device=dev)
     ws = moe.workspace(T, E, k, H, I, device=dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
@@ -508,9 +548,17 @@ def main(argv=None):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def fwd():
-        moe.moe_forward(x, logits, w13, w2, k, ws=ws, out=out, topk_ids=ids, topk_weights=wts,
-                        expert_offsets=off, permuted_rows=rows)
+    def fwd(events=None):
+        if e4m3:
+            moe.moe_forward_w8(x, logits, q13, s13, q2, s2, k, ws=ws, out=out, topk_ids=ids,
+                               topk_weights=wts, expert_offsets=off, permuted_rows=rows,
+                               events=events)
+        elif events is None:
+            moe.moe_forward(x, logits, w13, w2, k, ws=ws, out=out, topk_ids=ids,
+                            topk_weights=wts, expert_offsets=off, permuted_rows=rows)
+        else:
+            moe.moe_forward_timed(x, logits, w13, w2, k, events, ws=ws, out=out, topk_ids=ids,
+                                  topk_weights=wts, expert_offsets=off, permuted_rows=rows)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -559,10 +607,9 @@ def main(argv=None):
     barrier()
     for i in range(KB):
         flush.zero_()
-        moe.moe_forward_timed(x, logits, w13, w2, k, sev[i], ws=ws, out=out, topk_ids=ids,
-                              topk_weights=wts, expert_offsets=off, permuted_rows=rows)
+        fwd(sev[i])
     barrier()
-    fused = moe.moe_forward_fused(T, E, k, H, I)
+    fused = e4m3 or moe.moe_forward_fused(T, E, k, H, I)
     if fused:  # events 2..4 all follow the one FFN + combine launch
         spans = {"route_permute": (0, 1), "fused_ffn": (1, 4)}
     else:
@@ -596,21 +643,26 @@ def main(argv=None):
 
     # ---- roofline of the dominant kernel
     peaks, peak_kind = load_peaks()
-    work = stage_work(w, n_touched)
+    work = stage_work(w, n_touched, args.weights)
     dominant = max(stage_ms, key=lambda n: stage_ms[n])
     # The sustained bf16 peak was measured in a seconds-long loop under the 1 kW
     # power cap; it is the denominator when the timed steps ran under that cap too
     # (sw_power_cap seen while they ran) or lasted over a second.
     sustained = K * ms > 1000.0 or "sw_power_cap" in clocks.report()["reasons"]
     roof = roofline_entry(dominant, work[dominant], stage_ms[dominant], peaks, peak_kind,
-                          sustained, NCU_TRAFFIC.get((w.name, dominant)))
+                          sustained,
+                          NCU_TRAFFIC.get((w.name + ("+e4m3" if e4m3 else ""), dominant)))
     layer_bytes = work["w13"]["bytes"] + work["w2"]["bytes"] + work["route_permute"]["bytes"] + \
         work["combine"]["bytes"]
     layer_flops = work["w13"]["flops"] + work["w2"]["flops"]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        d_host = (wl.bf16_bits(x), logits.cpu().numpy(), wl.bf16_bits(w13), wl.bf16_bits(w2))
+        if e4m3:
+            d_host = (wl.bf16_bits(x), logits.cpu().numpy(),
+                      (q13.cpu().numpy(), s13.cpu().numpy()), (q2.cpu().numpy(), s2.cpu().numpy()))
+        else:
+            d_host = (wl.bf16_bits(x), logits.cpu().numpy(), wl.bf16_bits(w13), wl.bf16_bits(w2))
         import oracle
 
         v, sample, dt = oracle_sample(w, d_host, args.cpu_seconds)
@@ -618,7 +670,7 @@ def main(argv=None):
                "kind": "oracle", "sample": f"{sample} in {dt:.1f} s"}
 
     if rank == 0:
-        launches = moe.moe_forward_kernel_count(T, E, k, H, I)
+        launches = 2 if e4m3 else moe.moe_forward_kernel_count(T, E, k, H, I)
         line = {
             "metric": metric_name(w),
             "value": round(weak_scaling_value(world, T, ms), 2),

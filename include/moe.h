@@ -167,6 +167,37 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
                                  int32_t* expert_offsets, int32_t* permuted_rows,
                                  moe_stream_t stream);
 
+/* The layer with FP8 expert weights (the E4M3 format of "FP8 Formats for Deep
+ * Learning": sign, 4 exponent bits with bias 7, 3 significand bits, no
+ * infinities).  w13 uint8 [E, 2I, H] and w2 uint8 [E, H, I] hold E4M3 codes,
+ * w13_scale fp32 [E, 2I] and w2_scale fp32 [E, H] one scale per weight row:
+ * weight (e, r, c) = e4m3(code) * scale(e, r).  Everything else -- arguments,
+ * outputs, workspace (moe_workspace_size), routing, roundings, error reporting
+ * -- is moe_forward's.  The weights stream at one byte each and are widened to
+ * bf16 exactly in shared memory, so the tensor-core products are those of the
+ * bf16 path; each weight row's scale multiplies its fp32 accumulator row.  Runs
+ * only as the one-launch FFN (moe_forward_w8_supported; 2 kernels):
+ * MOE_ERR_UNSUPPORTED_SHAPE otherwise, whatever MOE_DISABLE_FUSED says.  Codes
+ * 0x7F / 0xFF (NaN) propagate as NaN.  All pointers 16-byte aligned. */
+moe_status_t moe_forward_w8(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
+                            const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                            moe_shape_t shape, moe_bf16_t* out, int32_t* topk_ids,
+                            float* topk_weights, int32_t* expert_offsets, int32_t* permuted_rows,
+                            void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward_w8 recording the 5 stage events of moe_forward_timed ([2] .. [4]
+ * all mark the end of the one FFN + combine launch). */
+moe_status_t moe_forward_w8_timed(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
+                                  const float* w13_scale, const uint8_t* w2,
+                                  const float* w2_scale, moe_shape_t shape, moe_bf16_t* out,
+                                  int32_t* topk_ids, float* topk_weights,
+                                  int32_t* expert_offsets, int32_t* permuted_rows,
+                                  void* workspace, size_t ws_bytes, moe_stream_t stream,
+                                  void* const* events, int n_events);
+
+/* 1 if moe_forward_w8 accepts `shape` (the one-launch FFN's shapes), else 0. */
+int moe_forward_w8_supported(moe_shape_t shape);
+
 /* Number of kernels one moe_forward call launches for `shape` (0 if unsupported). */
 int moe_forward_kernel_count(moe_shape_t shape);
 

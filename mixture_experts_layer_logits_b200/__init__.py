@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "MoeError", "Shape", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_forward_timed", "moe_forward_kernel_count",
-    "moe_forward_fused", "moe_selftest_wait_timeout",
+    "moe_forward_fused", "moe_forward_w8", "moe_forward_w8_supported", "moe_selftest_wait_timeout",
     "moe_device_status", "library_path", "load_library",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ERR_MISALIGNED",
     "MOE_ERR_WORKSPACE_TOO_SMALL", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
@@ -73,6 +73,13 @@ def load_library():
                                 ctypes.c_size_t, _vp]
     lib.moe_forward_timed.argtypes = [_vp, _vp, _vp, _vp, Shape, _vp, _vp, _vp, _vp, _vp, _vp,
                                       ctypes.c_size_t, _vp, ctypes.POINTER(_vp), ctypes.c_int]
+    lib.moe_forward_w8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, Shape, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, ctypes.c_size_t, _vp]
+    lib.moe_forward_w8_timed.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, Shape, _vp, _vp, _vp, _vp,
+                                         _vp, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_vp),
+                                         ctypes.c_int]
+    lib.moe_forward_w8_supported.argtypes = [Shape]
+    lib.moe_forward_w8_supported.restype = ctypes.c_int
     lib.moe_forward_kernel_count.argtypes = [Shape]
     lib.moe_forward_kernel_count.restype = ctypes.c_int
     lib.moe_forward_fused.argtypes = [Shape]
@@ -82,7 +89,8 @@ def load_library():
     lib.moe_selftest_wait_timeout.restype = ctypes.c_int
     lib.moe_device_status.argtypes = [_vp, ctypes.c_size_t, _vp]
     for fn in (lib.moe_route, lib.moe_permute, lib.moe_grouped_ffn, lib.moe_combine,
-               lib.moe_forward, lib.moe_forward_timed, lib.moe_device_status):
+               lib.moe_forward, lib.moe_forward_timed, lib.moe_forward_w8,
+               lib.moe_forward_w8_timed, lib.moe_device_status):
         fn.restype = ctypes.c_int
     lib.moe_status_string.argtypes = [ctypes.c_int]
     lib.moe_status_string.restype = ctypes.c_char_p
@@ -190,15 +198,19 @@ def moe_combine(y, topk_weights, out=None):
 
 
 def _forward(x, logits, w13, w2, top_k, ws, out, topk_ids, topk_weights, expert_offsets,
-             permuted_rows, events):
+             permuted_rows, events, scales=None):
     T, H = x.shape
     E = logits.shape[1]
     I = w13.shape[1] // 2
     dev = x.device
+    wdt = torch.bfloat16 if scales is None else torch.uint8
     _need(x, "x", torch.bfloat16, (T, H))
     _need(logits, "logits", torch.float32, (T, E))
-    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H))
-    _need(w2, "w2", torch.bfloat16, (E, H, I))
+    _need(w13, "w13", wdt, (E, 2 * I, H))
+    _need(w2, "w2", wdt, (E, H, I))
+    if scales is not None:
+        _need(scales[0], "w13_scale", torch.float32, (E, 2 * I))
+        _need(scales[1], "w2_scale", torch.float32, (E, H))
     if ws is None:
         ws = workspace(T, E, top_k, H, I, device=dev)
     if out is None:
@@ -210,14 +222,18 @@ def _forward(x, logits, w13, w2, top_k, ws, out, topk_ids, topk_weights, expert_
                              (permuted_rows, "permuted_rows", torch.int32, (T * top_k,))):
         if t is not None:
             _need(t, name, dt, shp)
-    args = (_ptr(x), _ptr(logits), _ptr(w13), _ptr(w2), Shape(T, E, top_k, H, I), _ptr(out),
+    weights = ((_ptr(w13), _ptr(w2)) if scales is None else
+               (_ptr(w13), _ptr(scales[0]), _ptr(w2), _ptr(scales[1])))
+    args = (_ptr(x), _ptr(logits), *weights, Shape(T, E, top_k, H, I), _ptr(out),
             _ptr(topk_ids), _ptr(topk_weights), _ptr(expert_offsets), _ptr(permuted_rows),
             _ptr(ws), ws.numel(), _stream(x))
+    lib = load_library()
+    name = "moe_forward" if scales is None else "moe_forward_w8"
     if events is None:
-        _check(load_library().moe_forward(*args), "moe_forward")
+        _check(getattr(lib, name)(*args), name)
     else:
         arr = (_vp * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
-        _check(load_library().moe_forward_timed(*args, arr, len(events)), "moe_forward_timed")
+        _check(getattr(lib, name + "_timed")(*args, arr, len(events)), name + "_timed")
     return out
 
 
@@ -236,6 +252,23 @@ def moe_forward_timed(x, logits, w13, w2, top_k: int, events, ws=None, out=None,
         raise ValueError("moe_forward_timed needs 5 events")
     return _forward(x, logits, w13, w2, top_k, ws, out, topk_ids, topk_weights, expert_offsets,
                     permuted_rows, events)
+
+
+def moe_forward_w8(x, logits, w13, w13_scale, w2, w2_scale, top_k: int, ws=None, out=None,
+                   topk_ids=None, topk_weights=None, expert_offsets=None, permuted_rows=None,
+                   events=None):
+    """The layer with FP8 (E4M3) expert weights: w13 / w2 uint8 codes [E, 2I, H] /
+    [E, H, I], w13_scale / w2_scale fp32 [E, 2I] / [E, H] (one scale per weight
+    row).  Other arguments and outputs as moe_forward; `events` (5
+    torch.cuda.Event, optional) as moe_forward_timed."""
+    if events is not None and len(events) != 5:
+        raise ValueError("moe_forward_w8 needs 5 events")
+    return _forward(x, logits, w13, w2, top_k, ws, out, topk_ids, topk_weights, expert_offsets,
+                    permuted_rows, events, scales=(w13_scale, w2_scale))
+
+
+def moe_forward_w8_supported(T: int, E: int, top_k: int, H: int, I: int) -> bool:
+    return bool(load_library().moe_forward_w8_supported(Shape(T, E, top_k, H, I)))
 
 
 def moe_forward_kernel_count(T: int, E: int, top_k: int, H: int, I: int) -> int:

@@ -46,6 +46,22 @@
 // weight tiles, evict-first), warp 1 TMEM allocator + MMA issuer, warps 2-7
 // gather (x rows for w13, act tiles for w2), warps 8-15 two epilogue groups,
 // then together the combine.
+//
+// FP8 weights (W8): w13 and w2 arrive as E4M3 codes with one fp32 scale per
+// weight row (weight = e4m3(q) * scale).  The producer streams the codes -- half
+// the bytes -- into their own ring, one [128 rows x 128 bytes] box per weight
+// block for every two K tiles.  Eight converter warps (3 of the bf16 kernel's
+// gather warps and four extra ones, 640 threads) widen each K tile to bf16 --
+// exact, every E4M3 value is a bf16 value -- and store it straight into tensor
+// memory, where the kind::f16 MMA takes its A operand (tcgen05.mma with A in
+// TMEM): with only 16 to 64 token columns, an A tile read from shared memory
+// would cost the MMA more than the whole stage's HBM time.  Warp 2 alone fills
+// the token operand into the B ring, its x-row copies arriving on the stage's
+// barrier as they land (cp.async.mbarrier.arrive) so it never waits on them.
+// The scale of a weight row is constant along K, so the epilogue multiplies
+// the fp32 accumulator row by it.
+#include <cuda_fp16.h>
+
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -72,6 +88,8 @@ struct FusedArgs {
     int32_t* w2_next;             // w2 units handed out at run time, zero at entry
     int32_t* split_out;           // [2] 1, S2 (CTA 0)
     int32_t* err;
+    const float* s13;             // W8: [E, 2I] w13 row scales
+    const float* s2;              // W8: [E, H] w2 row scales
     int k, H, I, R;
     int kt13, kt2;                // K tiles: H / 64, I / 64
     int fb13, fb2;                // I / 128 gate/up block pairs; ceil(H / 256) w2 block pairs
@@ -103,6 +121,70 @@ struct ComboScratch {
     float w[kMaxK];
 };
 
+// The FP8-weight kernel's buffers.  Shared memory after the 1 KB alignment
+// slack: B (kSB token tiles), then A8 (kS8 pair stages: two [128 x 128]-byte
+// E4M3 boxes in the 128-byte swizzle, K tiles kt and kt + 1, written by TMA);
+// then staging, Aux and the unit table as in the bf16 kernel.  A unit's K range
+// is always an even number of K tiles (H and I are multiples of 128, w2 slices
+// are rounded up to even lengths), so a pair stage never straddles two units.
+// Tensor memory (all 512 columns): accumulators in [0, 256), kSA converted A
+// stages in [256, 512), each two 128 x 64 bf16 tiles (row = lane, bf16 pairs
+// along 32 columns per tile).  Aux's barrier arrays are shared out in the order
+// A8, A, B.
+template <int NT>
+struct W8Cfg {
+    using C = Cfg<0, NT>;
+    static constexpr int kA8Bytes = 2 * kBM * 2 * kBK;
+    static constexpr int kBoxBytes = kBM * 2 * kBK;  // one [128 x 128]-byte box
+    static constexpr int kBBytes = C::kBTileBytes;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kNBuf = 256 / C::kAccCols;  // accumulator buffers: 8, 4, 2
+    static constexpr int kACol0 = 256;
+    static constexpr int kACols = 2 * kBK / 2;       // columns per converted stage
+    static constexpr int kSA = 256 / kACols;
+    static constexpr int kSB = NT <= 32 ? 6 : 4;
+    // The MMA frees A and B slots two K tiles at a time (one tcgen05.commit per
+    // pair: each commit drains the tensor pipe, about 200-300 cycles, as much as
+    // four of these M = 128, N <= 64 MMAs cost), so both rings have even depth
+    // and their "empty" barriers are per slot pair.
+    static_assert(kSA % 2 == 0 && kSB % 2 == 0, "slot pairs");
+    static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kUnitTableBytes;
+    static constexpr int kS8Raw = (C::kMaxSmem - kFixed - kSB * kBBytes) / kA8Bytes;
+    static constexpr int kS8 = kS8Raw < 16 - kSA - kSB ? kS8Raw : 16 - kSA - kSB;
+    static constexpr int kRingBytes = kSB * kBBytes + kS8 * kA8Bytes;
+    static constexpr int kSmemBytes = kFixed + kRingBytes;
+    static constexpr int kPf = 2;  // pair stages the producer prefetches into L2 ahead
+    // 640 threads: the roles of the bf16 kernel's warps 0..15, except that warps
+    // 4..7 convert the first box of each stage and the extra warps 16..19 the
+    // second (warp % 4 = the TMEM lane quarter, i.e. the 32 weight rows, it
+    // writes); warp 3 is idle
+    static constexpr int kThreads = 640;
+    static constexpr int kConv0 = 4, kConvExtra0 = 16, kConvWarps = 8;
+    // barrier slots in Aux's full/empty arrays
+    static constexpr int kBar8 = 0, kBarA = kS8, kBarB = kS8 + kSA;
+    static_assert(kS8 >= 3 && kS8 + kSA + kSB <= 16, "barrier slots");
+    static_assert(kSmemBytes <= C::kMaxSmem, "shared memory");
+    static_assert(kACol0 + kSA * kACols <= kTmemCols && kNBuf * C::kAccCols <= kACol0, "TMEM");
+};
+
+// Four E4M3 codes (byte i = element i) -> four bf16 values, two per word, lower
+// element in the lower half.  E4M3 -> f16 -> f32 -> bf16 are all exact for E4M3
+// values (3 significand bits, exponents 2^-9 .. 2^8), NaN stays NaN.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    uint32_t h0, h1;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(h0), "=r"(h1)
+        : "r"(w));
+    const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+    const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+    const __nv_bfloat162 b0 = __floats2bfloat162_rn(f0.x, f0.y);
+    const __nv_bfloat162 b1 = __floats2bfloat162_rn(f1.x, f1.y);
+    lo = *reinterpret_cast<const uint32_t*>(&b0);
+    hi = *reinterpret_cast<const uint32_t*>(&b1);
+}
+
 __device__ __forceinline__ void flag_error(int32_t* err, Aux* aux)
 {
     atomicExch(err, kDeviceErrorMagic);
@@ -127,18 +209,25 @@ __device__ __forceinline__ bool warp_wait_count(const int32_t* ctr, int target,
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+// W8: tm_w13 / tm_w2 map E4M3 codes ([128 x 64]-byte boxes, no swizzle).
+template <int NT, bool W8>
+__global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     fused_ffn_kernel(const __grid_constant__ CUtensorMap tm_w13,
                      const __grid_constant__ CUtensorMap tm_w2,
                      const __grid_constant__ CUtensorMap tm_act, const FusedArgs a)
 {
     using C = Cfg<0, NT>;
+    using R8 = W8Cfg<NT>;
     static_assert(NT <= 64, "weight-streaming tiles");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t* staging = ring + C::kStages * C::kStageBytes;
+    constexpr int kRingBytes = W8 ? R8::kRingBytes : C::kStages * C::kStageBytes;
+    constexpr int NBUF = W8 ? R8::kNBuf : C::kNBuf;  // accumulator buffers
+    constexpr int kTmemCols = W8 ? R8::kTmemCols : C::kTmemCols;
+    uint8_t* const bring = ring;                            // W8: token tiles
+    uint8_t* const ring8 = ring + R8::kSB * R8::kBBytes;    // W8: E4M3 pair stages
+    uint8_t* staging = ring + kRingBytes;
     Aux* aux = reinterpret_cast<Aux*>(staging + C::kStagingBytes);
     ComboScratch* combo = reinterpret_cast<ComboScratch*>(aux + 1);
     int* tok_off = reinterpret_cast<int*>(combo + 1);
@@ -148,11 +237,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&aux->full[s], 1 + C::kW);
-            mbar_init(&aux->empty[s], 1);
+        if constexpr (W8) {
+            for (int s = 0; s < R8::kS8; ++s) {
+                mbar_init(&aux->full[R8::kBar8 + s], 1);  // the producer's expect_tx
+                mbar_init(&aux->empty[R8::kBar8 + s], R8::kConvWarps);
+            }
+            for (int s = 0; s < R8::kSB; ++s) {
+                mbar_init(&aux->full[R8::kBarB + s], 1);  // the gather warp
+                mbar_init(&aux->empty[R8::kBarB + s], 1);  // empty: [0, kSB / 2), slot pairs
+            }
+            for (int s = 0; s < R8::kSA; ++s) {
+                // [0, kSA / 2): slot pairs
+                mbar_init(&aux->full[R8::kBarA + s], R8::kConvWarps);
+                mbar_init(&aux->empty[R8::kBarA + s], 1);
+            }
+        } else {
+            for (int s = 0; s < C::kStages; ++s) {
+                mbar_init(&aux->full[s], 1 + C::kW);
+                mbar_init(&aux->empty[s], 1);
+            }
         }
-        for (int b = 0; b < C::kNBuf; ++b) {
+        for (int b = 0; b < NBUF; ++b) {
             mbar_init(&aux->tfull[b], 1);
             mbar_init(&aux->tempty[b], 8);
         }
@@ -166,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_act);
     }
     if (warp == 1) {
-        tmem_alloc(&aux->tmem_base, C::kTmemCols);
+        tmem_alloc(&aux->tmem_base, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -186,7 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // slice adds epilogue publishes and combine reads (same-B200 A/B: 16 waves
     // 101.4 us decode / 360.7 us skewed decode, 4 waves 98.2 / 341.8).
     const int s2w = split_count(ntiles * a.fb2, a.s2_max, a.kt2, a.min_kt_per_split, 4);
-    const int ktps2 = (a.kt2 + s2w - 1) / s2w;
+    int ktps2 = (a.kt2 + s2w - 1) / s2w;
+    if (W8) ktps2 = (ktps2 + 1) & ~1;  // whole pair stages
     const int S2 = (a.kt2 + ktps2 - 1) / ktps2;  // every slice non-empty
     const int U13 = ntiles * a.fb13;
     const int U2 = ntiles * a.fb2 * S2;
@@ -264,7 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     // The CTA's i-th unit.  Dynamic entries live in the table as a ring with
     // tab_seq[slot] = i + 1 once published; no role trails the producer by more
-    // than kStages + kNBuf units, far below the ring's length.
+    // than its ring stages plus the accumulator buffers in units, far below the
+    // ring's length.
     auto get = [&](int i) {
         if (i < n_static) return i < kUnitTable ? read(i) : decode(unit_of(i));
         const int slot = i % kUnitTable;
@@ -289,10 +396,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();  // each weight block is read once
+            // W8: the E4M3 ring (its barriers are full/empty[0, kS8))
+            constexpr int NS = W8 ? R8::kS8 : C::kStages;
+            constexpr int kStBytes = W8 ? R8::kA8Bytes : C::kStageBytes;
+            constexpr int kBox1 = W8 ? kBM * 2 * kBK : kATileBytes;  // offset of the second box
+            constexpr int kKtStep = W8 ? 2 : 1;  // K tiles per ring stage
+            constexpr uint32_t kTx = W8 ? (uint32_t)R8::kA8Bytes : C::kTxBytes;
+            uint8_t* const pring = W8 ? ring8 : ring;
             int stage = 0;
             uint32_t phase = 0;
             int issued[16];
-            for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
+            for (int s = 0; s < NS; ++s) issued[s] = 0;
             bool ok = true;
             for (int i = 0; ok; ++i) {
                 Unit un;
@@ -320,18 +434,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int row0 = un.ph ? t.expert * a.H + un.fb * 2 * kBM
                                        : t.expert * 2 * a.I + un.fb * kBM;
                 const int row1 = un.ph ? row0 + kBM : row0 + a.I;
-                for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                if constexpr (W8) {
+                    // the E4M3 ring holds fewer bytes than the bf16 one: K tiles
+                    // kPf ahead of the TMA go to L2 now to keep as many weight
+                    // bytes in flight
+                    for (int kt = un.kt0 + 2; kt < min(un.kt1, un.kt0 + 2 * R8::kPf); kt += 2) {
+                        tma_prefetch_l2_2d(tm, kt * kBK, row0);
+                        tma_prefetch_l2_2d(tm, kt * kBK, row1);
+                    }
+                }
+                for (int kt = un.kt0; kt < un.kt1; kt += kKtStep) {
                     if (!mbar_wait(&aux->empty[stage], phase ^ 1u, abort_flag)) {
                         flag_error(a.err, aux);
                         ok = false;
                         break;
                     }
-                    uint8_t* st = ring + stage * C::kStageBytes;
-                    mbar_arrive_expect_tx(&aux->full[stage], C::kTxBytes);
+                    uint8_t* st = pring + stage * kStBytes;
+                    mbar_arrive_expect_tx(&aux->full[stage], kTx);
                     tma_load_2d(st, tm, &aux->full[stage], kt * kBK, row0, pol);
-                    tma_load_2d(st + kATileBytes, tm, &aux->full[stage], kt * kBK, row1, pol);
+                    tma_load_2d(st + kBox1, tm, &aux->full[stage], kt * kBK, row1, pol);
+                    if (W8 && kt + 2 * R8::kPf < un.kt1) {
+                        tma_prefetch_l2_2d(tm, (kt + 2 * R8::kPf) * kBK, row0);
+                        tma_prefetch_l2_2d(tm, (kt + 2 * R8::kPf) * kBK, row1);
+                    }
                     issued[stage] += 1;
-                    if (++stage == C::kStages) {
+                    if (++stage == NS) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -339,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok || *abort_flag) {
                 // let every TMA load already issued land before the CTA can exit
-                for (int s = 0; s < C::kStages; ++s)
+                for (int s = 0; s < NS; ++s)
                     if (issued[s] > 0) {
                         volatile int never = 0;
                         mbar_wait(&aux->full[s], (uint32_t)((issued[s] - 1) & 1), &never,
@@ -352,13 +479,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
+            int q = 0;  // W8: global stage number
             bool ok = true;
             for (int lu = 0; ok; ++lu) {
                 const Unit un = get(lu);
                 if (un.ph >= kUnitEnd) break;
                 const Unit& t = un;
-                const int b = lu % C::kNBuf;
-                const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
+                const int b = lu % NBUF;
+                const uint32_t aphase = (uint32_t)((lu / NBUF) & 1);
                 if (!mbar_wait(&aux->tempty[b], aphase ^ 1u, abort_flag)) {
                     flag_error(a.err, aux);
                     break;
@@ -368,26 +496,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t idesc = umma_idesc_bf16(kBM, n);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::kAccCols);
                 for (int kt = un.kt0; kt < un.kt1; ++kt) {
-                    if (!mbar_wait(&aux->full[stage], phase, abort_flag)) {
-                        flag_error(a.err, aux);
-                        ok = false;
-                        break;
+                    uint32_t st, bt;
+                    if constexpr (W8) {
+                        // A arrives a pair of K tiles at a time (slots 2 pa, 2 pa + 1)
+                        const int sa = q % R8::kSA, sb = q % R8::kSB;
+                        const int pa = (q >> 1) % (R8::kSA / 2);
+                        if (((q & 1) == 0 &&
+                             !mbar_wait(&aux->full[R8::kBarA + pa],
+                                        (uint32_t)(((q >> 1) / (R8::kSA / 2)) & 1), abort_flag)) ||
+                            !mbar_wait(&aux->full[R8::kBarB + sb], (uint32_t)((q / R8::kSB) & 1),
+                                       abort_flag)) {
+                            flag_error(a.err, aux);
+                            ok = false;
+                            break;
+                        }
+                        // the x rows of B were written by cp.async (generic proxy)
+                        fence_proxy_async_smem();
+                        st = tmem_base + R8::kACol0 + sa * R8::kACols;  // A in TMEM
+                        bt = smem_u32(bring + sb * R8::kBBytes);
+                    } else {
+                        if (!mbar_wait(&aux->full[stage], phase, abort_flag)) {
+                            flag_error(a.err, aux);
+                            ok = false;
+                            break;
+                        }
+                        st = smem_u32(ring + stage * C::kStageBytes);
+                        bt = st + C::kNA * kATileBytes;
                     }
                     tc_fence_after();
-                    const uint32_t st = smem_u32(ring + stage * C::kStageBytes);
-                    const uint32_t bt = st + C::kNA * kATileBytes;
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                         const uint32_t acc = (kt > un.kt0 || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
-                        umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
-                        umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
-                                  idesc, acc);
+                        if constexpr (W8) {  // K step kk: 8 columns of each converted tile
+                            umma_bf16_ts(d0, st + kk * (kUmmaK / 2), bdesc, idesc, acc);
+                            umma_bf16_ts(d0 + NT, st + R8::kACols / 2 + kk * (kUmmaK / 2), bdesc,
+                                         idesc, acc);
+                        } else {
+                            umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
+                            umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
+                                      idesc, acc);
+                        }
                     }
-                    umma_commit(&aux->empty[stage]);  // frees the smem stage when read
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
+                    if constexpr (W8) {  // free the A and B slot pairs when read
+                        if (q & 1) {
+                            umma_commit(&aux->empty[R8::kBarA + (q >> 1) % (R8::kSA / 2)]);
+                            umma_commit(&aux->empty[R8::kBarB + (q >> 1) % (R8::kSB / 2)]);
+                        }
+                        ++q;
+                    } else {
+                        umma_commit(&aux->empty[stage]);  // frees the smem stage when read
+                        if (++stage == C::kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
                     }
                 }
                 if (ok) umma_commit(&aux->tfull[b]);
@@ -397,9 +559,143 @@ __global__ void __launch_bounds__(kThreads, 1)
             volatile int never = 0;
             if (!mbar_wait(&aux->drain, 0, &never, 500000000ull)) atomicExch(a.err, kDeviceErrorMagic);
         }
+    } else if (W8 && warp == 2) {
+        // ------------------------------------------------------------ token operand (W8)
+        // One warp fills the B ring: x rows by cp.async, each lane's copies arriving
+        // on the stage's barrier when they land, or one act TMA.  Nothing here waits
+        // for its own copies, so the ring runs kSB stages ahead of the MMA.
+        int* my_off = tok_off;
+        const uint64_t keep = l2_policy_evict_last();  // x / act rows are re-read per block
+        int q = 0;
+        int cur_tile = -1, cur_ph = -1, ready_tile = -1;
+        int last_tma[R8::kSB];  // stage of each slot's latest use when that was a TMA, else -1
+        for (int sb = 0; sb < R8::kSB; ++sb) last_tma[sb] = -1;
+        bool ok = true;
+        for (int i = 0; ok; ++i) {
+            const Unit un = get(i);
+            if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
+            const Unit& t = un;
+            if (un.ph == 1 && un.tile != ready_tile) {
+                // every w13 unit of this tile has stored its act rows
+                if (!warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
+                    if (lane == 0) flag_error(a.err, aux);
+                    ok = false;
+                    break;
+                }
+                fence_proxy_async_global();  // the act TMA reads after the acquire
+                ready_tile = un.tile;
+            }
+            if (un.tile != cur_tile || un.ph != cur_ph) {
+                __syncwarp();  // earlier copies' addresses are all issued
+                if (un.ph == 0)
+                    for (int j = lane; j < t.rows; j += 32)
+                        my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
+                __syncwarp();
+                cur_tile = un.tile;
+                cur_ph = un.ph;
+            }
+            for (int kt = un.kt0; kt < un.kt1; ++kt, ++q) {
+                const int sb = q % R8::kSB, pb = (q >> 1) % (R8::kSB / 2);
+                uint64_t* fb = &aux->full[R8::kBarB + sb];
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&aux->empty[R8::kBarB + pb],
+                                          (uint32_t)((((q >> 1) / (R8::kSB / 2)) & 1) ^ 1),
+                                          abort_flag))) {
+                    if (lane == 0) flag_error(a.err, aux);
+                    ok = false;
+                    break;
+                }
+                uint8_t* btile = bring + sb * R8::kBBytes;
+                if (un.ph == 1) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, R8::kBBytes);
+                        tma_load_2d_nohint(btile, &tm_act, fb, 0, kt * a.R + t.row_start);
+                    }
+                    last_tma[sb] = q;
+                    continue;
+                }
+                last_tma[sb] = -1;
+                const uint32_t bt = smem_u32(btile);
+                const __nv_bfloat16* src0 = a.x + kt * kBK;
+                for (int c8 = lane; c8 < t.rows * 8; c8 += 32) {
+                    const int j = c8 >> 3, c = c8 & 7;
+                    cp_async_16_hint(bt + j * 128 + ((c ^ (j & 7)) << 4), src0 + my_off[j] + c * 8,
+                                     keep);
+                }
+                cp_async_mbar_arrive(fb);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(fb);
+            }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        if (lane == 0 && (!ok || *abort_flag)) {
+            // act TMAs still in flight land before the CTA can exit
+            for (int sb = 0; sb < R8::kSB; ++sb)
+                if (last_tma[sb] >= 0) {
+                    volatile int never = 0;
+                    mbar_wait(&aux->full[R8::kBarB + sb], (uint32_t)((last_tma[sb] / R8::kSB) & 1),
+                              &never, 500000000ull);
+                }
+        }
+    } else if (W8 && ((warp >= R8::kConv0 && warp < kEpiWarp0) || warp >= R8::kConvExtra0)) {
+        // ------------------------------------------------------------ converters (W8)
+        // Thread = weight row r = 32 (warp % 4) + lane of box `box` (gate / up, or
+        // the two w2 row blocks).  Per pair stage, for each of its two K tiles, it
+        // reads its row's 64 codes (four 16-byte chunks; in the 128-byte swizzle, 8
+        // consecutive rows put a chunk in 8 distinct bank groups, so the loads do
+        // not conflict), widens them to 32 bf16 pairs and stores them to 32 TMEM
+        // columns of lane r; then one arrival hands both K tiles to the MMA.
+        const int qd = warp & 3;
+        const int box = warp >= R8::kConvExtra0 ? 1 : 0;
+        const int r = qd * 32 + lane;
+        const uint32_t tst = tmem_base + ((uint32_t)(qd * 32) << 16) + R8::kACol0 +
+                             box * (R8::kACols / 2);
+        int q = 0;
+        bool ok = true;
+        for (int i = 0; ok; ++i) {
+            const Unit un = get(i);
+            if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
+            for (int kt = un.kt0; kt < un.kt1; kt += 2, q += 2) {  // one pair stage
+                const int pq = q >> 1, s8 = pq % R8::kS8, pa = pq % (R8::kSA / 2);
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&aux->empty[R8::kBarA + pa],
+                                          (uint32_t)(((pq / (R8::kSA / 2)) & 1) ^ 1), abort_flag)) ||
+                    !__all_sync(0xffffffffu, mbar_wait(&aux->full[R8::kBar8 + s8],
+                                                       (uint32_t)((pq / R8::kS8) & 1), abort_flag))) {
+                    if (lane == 0) flag_error(a.err, aux);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();  // the MMA that read these columns has completed
+                const uint8_t* src = ring8 + s8 * R8::kA8Bytes + box * R8::kBoxBytes + r * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // K tile kt + h: A slot 2 pa + h
+                    uint32_t o[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {  // K elements 16 c .. 16 c + 15 of the tile
+                        const uint4 v =
+                            *reinterpret_cast<const uint4*>(src + (((c + 4 * h) ^ (r & 7)) << 4));
+                        e4m3x4_to_bf16x4(v.x, o[8 * c + 0], o[8 * c + 1]);
+                        e4m3x4_to_bf16x4(v.y, o[8 * c + 2], o[8 * c + 3]);
+                        e4m3x4_to_bf16x4(v.z, o[8 * c + 4], o[8 * c + 5]);
+                        e4m3x4_to_bf16x4(v.w, o[8 * c + 6], o[8 * c + 7]);
+                    }
+                    tmem_st32(tst + (2 * pa + h) * R8::kACols, o);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&aux->full[R8::kBarA + pa]);
+                    mbar_arrive(&aux->empty[R8::kBar8 + s8]);  // pair stage read
+                }
+            }
+        }
     } else if (warp < 2 + kGatherWarps) {
         // ------------------------------------------------------------ gather
-        if (warp - 2 < C::kG * C::kW) {
+        // (W8: only warp 3 gets here, and it has nothing to do)
+        if (!W8 && warp - 2 < C::kG * C::kW) {
             constexpr int G = C::kG, W = C::kW;
             const int g = (warp - 2) / W, wi = (warp - 2) % W;
             int* my_off = tok_off + (warp - 2) * NT;
@@ -490,8 +786,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int lu = 0;; ++lu) {
             const Unit un = get(lu);
             const Unit& t = un;
-            const int b = lu % C::kNBuf;
-            const uint32_t aphase = (uint32_t)((lu / C::kNBuf) & 1);
+            const int b = lu % NBUF;
+            const uint32_t aphase = (uint32_t)((lu / NBUF) & 1);
+            // W8: this thread's two weight-row scales (gate and up rows, or output
+            // features f and f + 128), loaded before the accumulator wait
+            float sc0 = 1.f, sc1 = 1.f;
+            if constexpr (W8) {
+                if (un.ph == 0) {
+                    const float* sp = a.s13 + (size_t)un.expert * 2 * a.I + un.fb * kBM + f_local;
+                    sc0 = __ldg(sp);
+                    sc1 = __ldg(sp + a.I);
+                } else if (un.ph == 1) {
+                    const int f2 = un.fb * 2 * kBM + f_local;
+                    const float* sp = a.s2 + (size_t)un.expert * a.H + f2;
+                    sc0 = __ldg(sp);
+                    if (f2 + kBM < a.H) sc1 = __ldg(sp + kBM);
+                }
+            }
             bool got = false;
             if (un.ph < kUnitEnd) {
                 got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
@@ -523,6 +834,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld8(tacc + j0, gv);
                     tmem_ld8(tacc + NT + j0, vv);
                     tmem_ld_wait();
+                    if constexpr (W8) {
+#pragma unroll
+                        for (int jj = 0; jj < kStageRows; ++jj) {
+                            gv[jj] = __float_as_uint(__uint_as_float(gv[jj]) * sc0);
+                            vv[jj] = __float_as_uint(__uint_as_float(vv[jj]) * sc1);
+                        }
+                    }
                     if (j0 + kStageRows >= jend) {  // accumulator drained: let the MMA go on
                         tc_fence_before();
                         __syncwarp();
@@ -569,8 +887,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         {  // w2 slice: fp32 by expanded id
                             const int r = a.permuted_rows[p];
                             float* prow = a.part2 + ((size_t)un.split * a.R + r) * a.H;
-                            prow[f] = __uint_as_float(gv[jj]);
-                            if (f1_ok) prow[f + kBM] = __uint_as_float(vv[jj]);
+                            float g0 = __uint_as_float(gv[jj]), g1 = __uint_as_float(vv[jj]);
+                            if constexpr (W8) {
+                                g0 *= sc0;
+                                g1 *= sc1;
+                            }
+                            prow[f] = g0;
+                            if (f1_ok) prow[f + kBM] = g1;
                         }
                     }
                 }
@@ -661,11 +984,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
-template <int NT>
+template <int NT, bool W8>
 cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const CUtensorMap& ta,
                             const FusedArgs& a, int grid, cudaStream_t st)
 {
@@ -674,14 +997,14 @@ cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const
     // table follows the aux area
     static_assert(sizeof(Aux) + sizeof(ComboScratch) <= 1024, "aux area");
     static_assert(C::kAuxBytes % 16 == 0, "unit table alignment");
-    constexpr int smem = C::kSmemBytes + kUnitTableBytes;
+    constexpr int smem = W8 ? W8Cfg<NT>::kSmemBytes : C::kSmemBytes + kUnitTableBytes;
     static_assert(smem <= C::kMaxSmem, "shared memory");
-    auto kern = fused_ffn_kernel<NT>;
+    auto kern = fused_ffn_kernel<NT, W8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(W8 ? W8Cfg<NT>::kThreads : kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -711,9 +1034,14 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
                              const FfnPlan& plan, cudaStream_t st)
 {
     const int R = T * k;
+    const bool w8 = b.s13 != nullptr;
     CUtensorMap t13, t2, ta;
-    cudaError_t err = make_tmap(&t13, b.w13, (uint64_t)E * 2 * I, (uint64_t)H, kBM);
-    if (err == cudaSuccess) err = make_tmap(&t2, b.w2, (uint64_t)E * H, (uint64_t)I, kBM);
+    // E4M3 codes: [128 rows x 128 bytes] boxes (two K tiles), 128-byte swizzle
+    cudaError_t err = w8 ? make_tmap_u8(&t13, b.w13, (uint64_t)E * 2 * I, (uint64_t)H, kBM, 2 * kBK)
+                         : make_tmap(&t13, b.w13, (uint64_t)E * 2 * I, (uint64_t)H, kBM);
+    if (err == cudaSuccess)
+        err = w8 ? make_tmap_u8(&t2, b.w2, (uint64_t)E * H, (uint64_t)I, kBM, 2 * kBK)
+                 : make_tmap(&t2, b.w2, (uint64_t)E * H, (uint64_t)I, kBM);
     // act, K-blocked: (I / 64) * R rows of 64 columns, NT-row boxes
     if (err == cudaSuccess)
         err = make_tmap(&ta, b.act, (uint64_t)(I / kBK) * R, (uint64_t)kBK, (uint32_t)plan.nt);
@@ -743,10 +1071,15 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     a.fb2 = (H / kBM + 1) / 2;
     a.s2_max = plan.s2_max;
     a.min_kt_per_split = 4;
-    switch (plan.nt) {
-    case 16: return launch_fused_nt<16>(t13, t2, ta, a, plan.grid, st);
-    case 32: return launch_fused_nt<32>(t13, t2, ta, a, plan.grid, st);
-    case 64: return launch_fused_nt<64>(t13, t2, ta, a, plan.grid, st);
+    a.s13 = b.s13;
+    a.s2 = b.s2;
+    switch (plan.nt * 2 + (w8 ? 1 : 0)) {
+    case 32: return launch_fused_nt<16, false>(t13, t2, ta, a, plan.grid, st);
+    case 64: return launch_fused_nt<32, false>(t13, t2, ta, a, plan.grid, st);
+    case 128: return launch_fused_nt<64, false>(t13, t2, ta, a, plan.grid, st);
+    case 33: return launch_fused_nt<16, true>(t13, t2, ta, a, plan.grid, st);
+    case 65: return launch_fused_nt<32, true>(t13, t2, ta, a, plan.grid, st);
+    case 129: return launch_fused_nt<64, true>(t13, t2, ta, a, plan.grid, st);
     default: return cudaErrorInvalidValue;
     }
 }

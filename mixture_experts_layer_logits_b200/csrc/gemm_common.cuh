@@ -188,5 +188,25 @@ inline cudaError_t make_tmap(CUtensorMap* m, const void* base, uint64_t rows, ui
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 2D byte tensor (E4M3 weight codes) [rows, cols] with a [box_rows, box_cols] box:
+// box_cols 64 unswizzled, or 128 with the 128-byte swizzle (16-byte chunk c of box
+// row r lands at chunk c ^ (r % 8) of its 128-byte shared-memory row).
+inline cudaError_t make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                                uint32_t box_rows, uint32_t box_cols = kBK)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    if (box_cols != 64 && box_cols != 128) return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          box_cols == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace gemm
 }  // namespace moe

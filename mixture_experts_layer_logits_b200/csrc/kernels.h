@@ -105,8 +105,10 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
 // weight-streaming shapes: at most 64 tokens, so every expert's rows fit one tile.
 struct FusedBuffers {
     const void* x;
-    const void* w13;
+    const void* w13;   // bf16 weights, or E4M3 codes when s13 is set
     const void* w2;
+    const float* s13;  // E4M3 weights: [E, 2I] and [E, H] fp32 row scales; else nullptr
+    const float* s2;
     const int32_t* permuted_rows;
     const Tile* tiles;
     const int32_t* num_tiles;

@@ -167,11 +167,13 @@ PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
     return a;
 }
 
-// w13_prefetch: for the one-launch FFN, the w13 weights whose first K tiles the
-// permutation kernel prefetches into L2 (single-CTA path only).
+// w13_prefetch: for the one-launch FFN, the w13 weights (bf16, or E4M3 codes when
+// prefetch_e4m3) whose first K tiles the permutation kernel prefetches into L2
+// (single-CTA path only).
 moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, const moe_shape_t& s,
                          int32_t* offsets, int32_t* rows, void* ws, const Layout& L,
-                         cudaStream_t st, const void* w13_prefetch = nullptr)
+                         cudaStream_t st, const void* w13_prefetch = nullptr,
+                         bool prefetch_e4m3 = false)
 {
     PermuteAux aux = make_aux(ws, L, s);
     const long R = (long)s.T * s.top_k;
@@ -179,8 +181,11 @@ moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, cons
     if (R <= kSmallRows) {
         CUtensorMap pf;
         const CUtensorMap* pf_map = nullptr;
+        const uint64_t pf_rows = (uint64_t)s.E * 2 * s.I;
         if (w13_prefetch &&
-            gemm::make_tmap(&pf, w13_prefetch, (uint64_t)s.E * 2 * s.I, (uint64_t)s.H, gemm::kBM) ==
+            (prefetch_e4m3
+                 ? gemm::make_tmap_u8(&pf, w13_prefetch, pf_rows, (uint64_t)s.H, gemm::kBM)
+                 : gemm::make_tmap(&pf, w13_prefetch, pf_rows, (uint64_t)s.H, gemm::kBM)) ==
                 cudaSuccess) {
             pf_map = &pf;
             // each fused CTA's first w13 unit, as far as there can be w13 units:
@@ -192,7 +197,8 @@ moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, cons
             // 16 K tiles (2 x 128 x 1024 weights per CTA) cover the routing and
             // fused-kernel set-up window; 8 left HBM idle part of it, 20 and 24
             // gained nothing more (same-B200 A/B)
-            constexpr int kPrefetchKt = 16;
+            // (E4M3 codes: the same bytes are twice the K tiles)
+            const int kPrefetchKt = prefetch_e4m3 ? 32 : 16;
             aux.pf_kt = s.H / gemm::kBK < kPrefetchKt ? s.H / gemm::kBK : kPrefetchKt;
         }
         e = launch_small_route_permute(logits, s.T, s.E, s.top_k, ids, weights, offsets, rows, aux,
@@ -298,14 +304,18 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
                                       static_cast<cudaStream_t>(stream)));
 }
 
-static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
-                                 const moe_bf16_t* w2, moe_shape_t s, moe_bf16_t* out,
-                                 int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
-                                 int32_t* permuted_rows, void* ws, size_t ws_bytes,
-                                 moe_stream_t stream, void* const* events)
+// s13 / s2 set: w13 / w2 are E4M3 codes with those row scales (one-launch path only).
+static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const void* w13,
+                                 const void* w2, const float* s13, const float* s2, moe_shape_t s,
+                                 moe_bf16_t* out, int32_t* topk_ids, float* topk_weights,
+                                 int32_t* expert_offsets, int32_t* permuted_rows, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream, void* const* events)
 {
-    if (!x || !logits || !w13 || !w2 || !out || !ws) return MOE_ERR_INVALID_ARG;
+    const bool w8 = s13 || s2;
+    if (!x || !logits || !w13 || !w2 || !out || !ws || (w8 && !(s13 && s2)))
+        return MOE_ERR_INVALID_ARG;
     if (!ffn_shape_ok(s)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (w8 && (!aligned16(s13) || !aligned16(s2))) return MOE_ERR_MISALIGNED;
     if (!aligned16(x) || !aligned16(logits) || !aligned16(w13) || !aligned16(w2) ||
         !aligned16(out) || !aligned16(ws) || (topk_ids && !aligned16(topk_ids)) ||
         (topk_weights && !aligned16(topk_weights)) ||
@@ -325,9 +335,12 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
         return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st));
     };
 
-    const bool fused = L.fused && fused_enabled();
+    // E4M3 weights exist only on the one-launch path
+    if (w8 && !L.fused) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const bool fused = w8 || (L.fused && fused_enabled());
     moe_status_t r = mark(0);
-    if (r == MOE_OK) r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st, fused ? w13 : nullptr);
+    if (r == MOE_OK)
+        r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st, fused ? w13 : nullptr, w8);
     if (r == MOE_OK) r = mark(1);
     if (fused) {
         // one launch: w13, w2 and the combine (the stage events in between all
@@ -336,6 +349,8 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
         b.x = x;
         b.w13 = w13;
         b.w2 = w2;
+        b.s13 = s13;
+        b.s2 = s2;
         b.permuted_rows = rows;
         b.tiles = at<Tile>(ws, L.tiles);
         b.num_tiles = at<int32_t>(ws, L.num_tiles);
@@ -373,8 +388,8 @@ moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf1
                          float* topk_weights, int32_t* expert_offsets, int32_t* permuted_rows,
                          void* ws, size_t ws_bytes, moe_stream_t stream)
 {
-    return forward_impl(x, logits, w13, w2, s, out, topk_ids, topk_weights, expert_offsets,
-                        permuted_rows, ws, ws_bytes, stream, nullptr);
+    return forward_impl(x, logits, w13, w2, nullptr, nullptr, s, out, topk_ids, topk_weights,
+                        expert_offsets, permuted_rows, ws, ws_bytes, stream, nullptr);
 }
 
 moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
@@ -386,8 +401,39 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
     if (!events || n_events != 5) return MOE_ERR_INVALID_ARG;
     for (int i = 0; i < 5; ++i)
         if (!events[i]) return MOE_ERR_INVALID_ARG;
-    return forward_impl(x, logits, w13, w2, s, out, topk_ids, topk_weights, expert_offsets,
-                        permuted_rows, ws, ws_bytes, stream, events);
+    return forward_impl(x, logits, w13, w2, nullptr, nullptr, s, out, topk_ids, topk_weights,
+                        expert_offsets, permuted_rows, ws, ws_bytes, stream, events);
+}
+
+moe_status_t moe_forward_w8(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
+                            const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                            moe_shape_t s, moe_bf16_t* out, int32_t* topk_ids,
+                            float* topk_weights, int32_t* expert_offsets, int32_t* permuted_rows,
+                            void* ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!w13_scale || !w2_scale) return MOE_ERR_INVALID_ARG;
+    return forward_impl(x, logits, w13, w2, w13_scale, w2_scale, s, out, topk_ids, topk_weights,
+                        expert_offsets, permuted_rows, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status_t moe_forward_w8_timed(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
+                                  const float* w13_scale, const uint8_t* w2,
+                                  const float* w2_scale, moe_shape_t s, moe_bf16_t* out,
+                                  int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
+                                  int32_t* permuted_rows, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream, void* const* events, int n_events)
+{
+    if (!events || n_events != 5 || !w13_scale || !w2_scale) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i)
+        if (!events[i]) return MOE_ERR_INVALID_ARG;
+    return forward_impl(x, logits, w13, w2, w13_scale, w2_scale, s, out, topk_ids, topk_weights,
+                        expert_offsets, permuted_rows, ws, ws_bytes, stream, events);
+}
+
+int moe_forward_w8_supported(moe_shape_t s)
+{
+    if (!ffn_shape_ok(s)) return 0;
+    return layout_for(s).fused ? 1 : 0;
 }
 
 int moe_forward_kernel_count(moe_shape_t s)

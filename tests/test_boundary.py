@@ -136,6 +136,43 @@ def test_forward_validation(lib):
     assert lib.moe_forward(*args) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
 
 
+def test_forward_w8_validation(lib):
+    n = lib.moe_workspace_size(S())
+    ok = [A, A, A, A, A, A, S(), A, NUL, NUL, NUL, NUL, A, n, None]
+    for i in (0, 1, 2, 3, 4, 5, 7, 12):
+        args = list(ok)
+        args[i] = NUL
+        assert lib.moe_forward_w8(*args) == moe.MOE_ERR_INVALID_ARG
+    for i in (0, 1, 2, 3, 4, 5, 7, 12, 8, 9, 10, 11):
+        args = list(ok)
+        args[i] = MIS
+        assert lib.moe_forward_w8(*args) == moe.MOE_ERR_MISALIGNED
+    args = list(ok)
+    args[6] = S(H=130)
+    assert lib.moe_forward_w8(*args) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    args = list(ok)
+    args[13] = 0
+    assert lib.moe_forward_w8(*args) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    # FP8 weights run only as the one-launch FFN: T = 65 is refused before any launch
+    args = list(ok)
+    args[6] = S(T=65)
+    args[13] = lib.moe_workspace_size(S(T=65))
+    assert lib.moe_forward_w8(*args) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    ev = (ctypes.c_void_p * 5)(*([A] * 5))
+    assert lib.moe_forward_w8_timed(*ok, ev, 4) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_w8_timed(*ok, None, 5) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_forward_w8_supported(lib):
+    f = lib.moe_forward_w8_supported
+    assert f(S()) == 1                              # decode
+    assert f(S(T=64, E=256, H=7168, I=2048)) == 1   # skewed decode
+    assert f(S(T=16, E=8, k=2, H=256, I=512)) == 1  # tiny
+    assert f(S(T=65)) == 0
+    assert f(S(T=8192, H=4096, I=1536)) == 0        # prefill
+    assert f(S(H=100)) == 0
+
+
 def test_device_status_validation(lib):
     assert lib.moe_device_status(NUL, 1024, None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_device_status(A, 0, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
