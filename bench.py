@@ -48,7 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (workload, kernel), from the summaries under profiles/.  An entry is removed
 # when its kernel changes, until it is captured again.
 NCU_TRAFFIC = {
-    ("decode", "fused_ffn"): 509_732_864 + 3_883_776,  # profiles/fused_ffn_decode.md
+    ("decode", "fused_ffn"): 509_740_032 + 4_323_328,  # profiles/fused_ffn_decode.md
+    ("decode+e4m3", "fused_ffn"): 257_047_040 + 3_710_976,  # profiles/fused_ffn_w8_decode.md
     # profiles/grouped_gemm_prefill_shape.md: the 16-expert capture x 8
     ("prefill", "w13"): 3_510_591_488,
     ("prefill", "w2"): 2_175_619_072,
