@@ -50,12 +50,13 @@
 // FP8 weights (W8): w13 and w2 arrive as E4M3 codes with one fp32 scale per
 // weight row (weight = e4m3(q) * scale).  The producer streams the codes -- half
 // the bytes -- into their own ring, one [128 rows x 128 bytes] box per weight
-// block for every two K tiles.  Eight converter warps (3 of the bf16 kernel's
-// gather warps and four extra ones, 640 threads) widen each K tile to bf16 --
-// exact, every E4M3 value is a bf16 value -- and store it straight into tensor
-// memory, where the kind::f16 MMA takes its A operand (tcgen05.mma with A in
-// TMEM): with only 16 to 64 token columns, an A tile read from shared memory
-// would cost the MMA more than the whole stage's HBM time.  Warp 2 alone fills
+// block for every two K tiles.  Eight converter warps (warps 4-7 and four extra
+// warps 16-19, 640 threads) widen each K tile to bf16 -- exact, every E4M3 value
+// is a bf16 value -- and store it straight into tensor memory, where the
+// kind::f16 MMA takes its A operand (tcgen05.mma with A in TMEM).  That keeps
+// the bf16 tiles out of shared memory: no second ring there (its 64 KB go to the
+// code ring) and no shared-memory traffic for them, which the MMA's operand reads
+// and the converters would share.  Warp 2 alone fills
 // the token operand into the B ring, its x-row copies arriving on the stage's
 // barrier as they land (cp.async.mbarrier.arrive) so it never waits on them.
 // The scale of a weight row is constant along K, so the epilogue multiplies
