@@ -467,8 +467,6 @@ def routing_bench(args, w, rank, world, local, dev, pg):
             "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
             "config": dict(w.as_dict(), parallelism=f"replicas{world}",
-                           weights=("e4m3 codes + fp32 row scales (moe_forward_w8)" if e4m3
-                                    else "bf16"),
                            l2="flushed before every step (256 MiB write), outside the step events"),
             "roofline": roof,
             "stage_ms": {"route": round(route_ms, 5), "permute": round(perm_ms, 5)},
@@ -687,6 +685,8 @@ def main(argv=None):
             "dtype": "bf16",
             "data": "synthetic (seeded; weights N(0,1/sqrt(fan_in)) random-init)",
             "config": dict(w.as_dict(), parallelism=f"replicas{world}",
+                           weights=("e4m3 codes + fp32 row scales (moe_forward_w8)" if e4m3
+                                    else "bf16"),
                            tokens_per_rank=T, l2="flushed before every step (256 MiB write), "
                            "outside the step events", n_touched_experts=n_touched),
             "roofline": roof,
