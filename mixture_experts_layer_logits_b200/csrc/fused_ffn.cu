@@ -210,7 +210,7 @@ __device__ __forceinline__ bool warp_wait_count(const int32_t* ctr, int target,
     }
 }
 
-// W8: tm_w13 / tm_w2 map E4M3 codes ([128 x 64]-byte boxes, no swizzle).
+// W8: tm_w13 / tm_w2 map E4M3 codes ([128 x 128]-byte boxes, 128-byte swizzle).
 template <int NT, bool W8>
 __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     fused_ffn_kernel(const __grid_constant__ CUtensorMap tm_w13,
@@ -244,11 +244,10 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 mbar_init(&aux->empty[R8::kBar8 + s], R8::kConvWarps);
             }
             for (int s = 0; s < R8::kSB; ++s) {
-                mbar_init(&aux->full[R8::kBarB + s], 1);  // the gather warp
-                mbar_init(&aux->empty[R8::kBarB + s], 1);  // empty: [0, kSB / 2), slot pairs
+                mbar_init(&aux->full[R8::kBarB + s], 1);   // per stage: the gather warp
+                mbar_init(&aux->empty[R8::kBarB + s], 1);  // per slot pair (first kSB / 2)
             }
-            for (int s = 0; s < R8::kSA; ++s) {
-                // [0, kSA / 2): slot pairs
+            for (int s = 0; s < R8::kSA; ++s) {  // per slot pair (first kSA / 2 used)
                 mbar_init(&aux->full[R8::kBarA + s], R8::kConvWarps);
                 mbar_init(&aux->empty[R8::kBarA + s], 1);
             }
@@ -436,8 +435,8 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                                        : t.expert * 2 * a.I + un.fb * kBM;
                 const int row1 = un.ph ? row0 + kBM : row0 + a.I;
                 if constexpr (W8) {
-                    // the E4M3 ring holds fewer bytes than the bf16 one: K tiles
-                    // kPf ahead of the TMA go to L2 now to keep as many weight
+                    // the E4M3 ring holds fewer K tiles than the bf16 one: pair
+                    // stages kPf ahead of the TMA go to L2 now, to keep more weight
                     // bytes in flight
                     for (int kt = un.kt0 + 2; kt < min(un.kt1, un.kt0 + 2 * R8::kPf); kt += 2) {
                         tma_prefetch_l2_2d(tm, kt * kBK, row0);
