@@ -32,3 +32,22 @@ def test_bench_refers_only_to_defined_names():
 
 def test_graft_entry_refers_only_to_defined_names():
     assert _undefined_globals(os.path.join(ROOT, "__graft_entry__.py")) == []
+
+
+def test_stage_work_counts_e4m3_weights_at_one_byte_plus_row_scales():
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_logits_b200 import workloads as wl
+
+    w = wl.WORKLOADS["decode"]
+    n = 54
+    bf = bench.stage_work(w, n)
+    f8 = bench.stage_work(w, n, "e4m3")
+    T, k, H, I = w.T, w.k, w.H, w.I
+    rest = T * H * 2 + T * k * 8 + T * H * 2  # x, routing weights and rows, out
+    assert bf["fused_ffn"]["bytes"] == n * 3 * I * H * 2 + rest
+    assert f8["fused_ffn"]["bytes"] == n * (3 * I * H + (2 * I + H) * 4) + rest
+    assert f8["fused_ffn"]["flops"] == bf["fused_ffn"]["flops"]  # same bf16 products
+    assert f8["route_permute"] == bf["route_permute"] and f8["combine"] == bf["combine"]
