@@ -682,8 +682,8 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                         e4m3x4_to_bf16x4(v.w, o[8 * c + 6], o[8 * c + 7]);
                     }
                     tmem_st32(tst + (2 * pa + h) * R8::kACols, o);
-                    tmem_st_wait();
                 }
+                tmem_st_wait();  // both K tiles' stores
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
