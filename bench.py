@@ -182,7 +182,8 @@ class ClockSampler:
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index, period=0.01):
+    # 2 ms: the decode timed region lasts about 20 ms and should still get ~10 samples
+    def __init__(self, device_index, period=0.002):
         self.period = period
         self.samples = []
         self.reasons = set()
