@@ -49,6 +49,7 @@ def _load():
                                           ctypes.POINTER(_u16p), i, i, i, i, i, i, i, _i32p,
                                           _f64p]
     lib.oracle_e4m3_to_double.argtypes = [_u8p, ctypes.c_long, _f64p]
+    lib.oracle_round_to_bf16.argtypes = [_f64p, ctypes.c_long, _f64p]
     lib.oracle_forward_w8.argtypes = [_u16p, _f32p, _u8p, _f32p, _u8p, _f32p, i, i, i, i, i,
                                       _f64p, _i32p, _f32p, _i32p, _i32p]
     lib.oracle_forward_tokens_w8.argtypes = [_u16p, _f32p, ctypes.POINTER(_u8p),
@@ -58,6 +59,7 @@ def _load():
     lib.oracle_num_threads.argtypes = []
     for fn in (lib.oracle_num_threads, lib.oracle_route, lib.oracle_permute, lib.oracle_ffn, lib.oracle_combine,
                lib.oracle_forward, lib.oracle_forward_tokens, lib.oracle_e4m3_to_double,
+               lib.oracle_round_to_bf16,
                lib.oracle_forward_w8, lib.oracle_forward_tokens_w8):
         fn.restype = ctypes.c_int
     _lib = lib
@@ -199,6 +201,16 @@ def e4m3_to_float64(q):
     q = _c(q, np.uint8)
     out = np.empty(q.shape, np.float64)
     _check(_load().oracle_e4m3_to_double(_p(q, _u8p), q.size, _p(out, _f64p)), "e4m3_to_double")
+    return out
+
+
+def round_to_bf16(v):
+    """float64 values -> the nearest bf16 values (via fp32, round to nearest even at
+    both steps), returned as float64: the rounding of the diagnostic
+    ``round_intermediates`` mode."""
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.float64)
+    _check(_load().oracle_round_to_bf16(_p(v, _f64p), v.size, _p(out, _f64p)), "round_to_bf16")
     return out
 
 

@@ -47,7 +47,9 @@
  * SwiGLU MLP, and a dense all-experts masked loop; for the FP8 weights, the
  * E4M3 decoder against a library conversion of every code, bit equality with
  * the bf16 layer when the dequantised weights are bf16 values, and a dense
- * dequantise-then-multiply check).
+ * dequantise-then-multiply check; for the diagnostic bf16 rounding, the library
+ * float64 -> bfloat16 conversion on ties, subnormals and the overflow boundary,
+ * and a dense loop that rounds act and y with it).
  */
 #include <math.h>
 #include <omp.h>
@@ -88,7 +90,9 @@ static double bf16_to_double(uint16_t b)
     return (double)f;
 }
 
-/* double -> bf16 via fp32, both steps round-to-nearest-even.  Only used by the
+/* double -> bf16 via fp32, both steps round-to-nearest-even (ties to the even
+ * significand; a finite value past the largest bf16 by half an ulp or more
+ * becomes infinity; infinities and NaNs keep their class).  Only used by the
  * diagnostic `round_intermediates` mode. */
 static double round_to_bf16(double v)
 {
@@ -102,6 +106,14 @@ static double round_to_bf16(double v)
     u &= 0xffff0000u;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* Applies round_to_bf16 to n doubles (exported for the pins). */
+int oracle_round_to_bf16(const double* in, long n, double* out)
+{
+    if (!in || !out || n < 0) return -1;
+    for (long i = 0; i < n; ++i) out[i] = round_to_bf16(in[i]);
+    return 0;
 }
 
 /* ---- 1. route ------------------------------------------------------------ */

@@ -273,6 +273,87 @@ def test_forward_tokens_matches_forward():
         oracle.forward_tokens(x, logits, [None] * E, [None] * E, k, toks, I)
 
 
+def _f64_from_f32_bits(bits):
+    return np.asarray(bits, np.uint32).view(np.float32).astype(np.float64)
+
+
+def _bf16_rounding_cases():
+    """fp32 bit patterns around bf16 rounding boundaries, plus doubles outside fp32."""
+    highs = [0x3F80, 0x3F81, 0x4049, 0x404A, 0x0000, 0x0001, 0x0002, 0x007F, 0x0080, 0x0081,
+             0x7F7E, 0x7F7F, 0x1234, 0x5555]
+    lows = [0x0000, 0x0001, 0x7FFF, 0x8000, 0x8001, 0xFFFF]
+    bits = [(h << 16) | lo for h in highs for lo in lows]
+    bits += [b | 0x80000000 for b in bits]                  # the same, negative
+    v = _f64_from_f32_bits(bits).tolist()
+    v += [0.0, -0.0, math.inf, -math.inf, 1e300, -1e300, 1e-300, -1e-300,
+          1.0 + 2.0 ** -8 + 2.0 ** -30,                     # fp32 rounds it onto a bf16 tie
+          float(np.finfo(np.float32).max), 2.0 ** -149, 2.0 ** -133 * 1.5]
+    rng = np.random.default_rng(23)
+    v += (rng.standard_normal(20000) * np.exp2(rng.integers(-140, 128, 20000))).tolist()
+    return np.array(v, np.float64)
+
+
+def test_round_to_bf16_is_the_library_conversion():
+    """The diagnostic rounding equals torch's float64 -> bfloat16 conversion (which
+    also goes through fp32 with round-to-nearest-even) bit for bit, on ties with
+    even and odd last significand bits, one fp32 ulp either side of a tie,
+    subnormals, the overflow boundary, signed zeros, infinities and a random
+    spread of magnitudes."""
+    v = _bf16_rounding_cases()
+    got = oracle.round_to_bf16(v)
+    want = torch.tensor(v).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(got.view(np.uint64), want.view(np.uint64))
+    # NaNs stay NaN, whatever their payload (an all-ones payload must not carry
+    # into the sign bit)
+    nans = np.array([0x7FF8000000000000, 0x7FFFFFFFFFFFFFFF, 0xFFFFFFFFFFFFFFFF,
+                     0x7FF0000000000001], np.uint64).view(np.float64)
+    assert np.isnan(oracle.round_to_bf16(nans)).all()
+
+
+def test_round_to_bf16_closed_forms():
+    """Values fixed by the definition of round-to-nearest-even on an 8-bit significand."""
+    ulp1 = 2.0 ** -7                      # bf16 spacing in [1, 2)
+    bf16_max = (2.0 - ulp1) * 2.0 ** 127
+    cases = [
+        (1.0 + ulp1 / 2, 1.0),                        # tie, even neighbour below
+        (1.0 + 3 * ulp1 / 2, 1.0 + 2 * ulp1),         # tie, even neighbour above
+        (1.0 + ulp1 / 2 + 2.0 ** -20, 1.0 + ulp1),    # just past the tie
+        (1.0 + ulp1 / 2 - 2.0 ** -20, 1.0),           # just short of it
+        (-(1.0 + 3 * ulp1 / 2), -(1.0 + 2 * ulp1)),
+        (bf16_max + 2.0 ** 119, math.inf),            # half an ulp past the largest: tie to inf
+        (bf16_max + 2.0 ** 118, bf16_max),
+        (2.0 ** -134, 0.0),                           # subnormal tie: 0 (even) and 2^-133 (odd)
+        (3 * 2.0 ** -134, 2.0 ** -132),               # tie between 2^-133 (odd) and 2^-132 (even)
+        (2.0 ** -135, 0.0),
+    ]
+    for v, want in cases:
+        got = float(oracle.round_to_bf16(np.array([v]))[0])
+        assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), (v, got, want)
+
+
+def test_round_intermediates_dense_loop():
+    """round_intermediates = True against a dense all-experts loop that rounds act
+    and y to bf16 with the library conversion (no permutation, no gather)."""
+    rng = np.random.default_rng(29)
+    T, E, k, H, I = 7, 5, 2, 16, 8
+    logits, x, w13, w2 = _rand_layer(rng, T, E, k, H, I)
+    res = oracle.forward(x, logits, w13, w2, k, round_intermediates=True)
+    ids, w = res["topk_ids"], res["topk_weights"]
+    X, W13, W2 = _bits_to_f64(x), _bits_to_f64(w13), _bits_to_f64(w2)
+    bf = lambda a: torch.tensor(a).to(torch.bfloat16).double().numpy()
+    dense = np.zeros((T, H))
+    for t in range(T):
+        for e in range(E):
+            hit = np.nonzero(ids[t] == e)[0]
+            m = float(w[t, hit[0]]) if len(hit) else 0.0
+            h = W13[e] @ X[t]
+            g, u = h[:I], h[I:]
+            dense[t] += m * bf(W2[e] @ bf(g / (1.0 + np.exp(-g)) * u))
+    np.testing.assert_allclose(res["out"], dense, rtol=1e-12, atol=1e-13)
+    exact = oracle.forward(x, logits, w13, w2, k)["out"]
+    assert not np.array_equal(res["out"], exact)
+
+
 def test_round_intermediates_stays_within_bf16_error():
     rng = np.random.default_rng(21)
     T, E, k, H, I = 8, 4, 2, 64, 32
@@ -435,6 +516,15 @@ MUTATIONS = [
     ("FP8 gate and up scales swapped",
      "const double sg = s13_e[c], su = s13_e[I + c];",
      "const double sg = s13_e[I + c], su = s13_e[c];"),
+    ("bf16 rounding truncates",
+     "u += 0x7fffu + lsb;",
+     "(void)lsb;"),
+    ("bf16 rounding ties away from zero",
+     "u += 0x7fffu + lsb;",
+     "u += 0x8000u; (void)lsb;"),
+    ("bf16 rounding drops the finite test (NaN/inf carry)",
+     "if ((u & 0x7f800000u) != 0x7f800000u) {          /* finite */",
+     "if (1) {"),
 ]
 
 
@@ -459,7 +549,10 @@ def test_planted_mistake_is_caught(name, old, new, monkeypatch, tmp_path):
                       lambda: test_permute_brute_force_and_invariants(33, 5, 3),
                       lambda: test_dense_masked_all_experts_loop(5, 6, 3, 8, 4),
                       test_e4m3_decoder_is_the_library_conversion,
-                      lambda: test_w8_dense_dequantised_loop(5, 6, 3, 8, 4)):
+                      lambda: test_w8_dense_dequantised_loop(5, 6, 3, 8, 4),
+                      test_round_to_bf16_is_the_library_conversion,
+                      test_round_to_bf16_closed_forms,
+                      test_round_intermediates_dense_loop):
             try:
                 check()
             except AssertionError:
