@@ -369,11 +369,19 @@ int oracle_forward_tokens(const uint16_t* x, const float* logits,
 
 /* ---- FP8 weights ------------------------------------------------------------ */
 
+/* dec[q] = e4m3_to_double(q) for all 256 codes: the decoder's values, looked up
+ * instead of recomputed for every weight. */
+static void e4m3_table(double* dec)
+{
+    for (int q = 0; q < 256; ++q) dec[q] = e4m3_to_double((uint8_t)q);
+}
+
 /* As expert_ffn_row with w13_e = [2I, H] E4M3 codes and s13_e = [2I] row scales,
- * w2_e = [H, I] codes and s2_e = [H] row scales: weight (r, c) = e4m3(q) * s[r]. */
+ * w2_e = [H, I] codes and s2_e = [H] row scales: weight (r, c) = e4m3(q) * s[r],
+ * with e4m3(q) = dec[q] (e4m3_table). */
 static void expert_ffn_row_w8(const uint16_t* x_row, const uint8_t* q13_e, const float* s13_e,
-                              const uint8_t* q2_e, const float* s2_e, int H, int I, double* act,
-                              double* y_row)
+                              const uint8_t* q2_e, const float* s2_e, int H, int I,
+                              const double* dec, double* act, double* y_row)
 {
     for (int c = 0; c < I; ++c) {
         const uint8_t* qg = q13_e + (size_t)c * H;
@@ -382,8 +390,8 @@ static void expert_ffn_row_w8(const uint16_t* x_row, const uint8_t* q13_e, const
         double gate = 0.0, up = 0.0;
         for (int i = 0; i < H; ++i) {
             const double xi = bf16_to_double(x_row[i]);
-            gate += xi * (e4m3_to_double(qg[i]) * sg);
-            up += xi * (e4m3_to_double(qu[i]) * su);
+            gate += xi * (dec[qg[i]] * sg);
+            up += xi * (dec[qu[i]] * su);
         }
         act[c] = gate / (1.0 + exp(-gate)) * up;
     }
@@ -391,7 +399,7 @@ static void expert_ffn_row_w8(const uint16_t* x_row, const uint8_t* q13_e, const
         const uint8_t* q = q2_e + (size_t)o * I;
         const double so = s2_e[o];
         double acc = 0.0;
-        for (int c = 0; c < I; ++c) acc += act[c] * (e4m3_to_double(q[c]) * so);
+        for (int c = 0; c < I; ++c) acc += act[c] * (dec[q[c]] * so);
         y_row[o] = acc;
     }
 }
@@ -411,6 +419,8 @@ int oracle_forward_w8(const uint16_t* x, const float* logits, const uint8_t* q13
     const long R = (long)T * k;
     double* y = (double*)malloc(sizeof(double) * (size_t)R * H);
     if (!y) return -2;
+    double dec[256];
+    e4m3_table(dec);
     int bad = 0;
 #pragma omp parallel
     {
@@ -425,7 +435,7 @@ int oracle_forward_w8(const uint16_t* x, const float* logits, const uint8_t* q13
                     const long r = permuted_rows[p];
                     expert_ffn_row_w8(x + (size_t)(r / k) * H, q13 + (size_t)e * 2 * I * H,
                                       s13 + (size_t)e * 2 * I, q2 + (size_t)e * H * I,
-                                      s2 + (size_t)e * H, H, I, act, y + (size_t)r * H);
+                                      s2 + (size_t)e * H, H, I, dec, act, y + (size_t)r * H);
                 }
             }
             free(act);
@@ -449,6 +459,8 @@ int oracle_forward_tokens_w8(const uint16_t* x, const float* logits,
     if (T < 1 || E < 1 || k < 1 || k > E || H < 1 || I < 1 || n_sel < 0) return -1;
     for (int s = 0; s < n_sel; ++s)
         if (tokens[s] < 0 || tokens[s] >= T) return -1;
+    double dec[256];
+    e4m3_table(dec);
     int bad = 0;
 #pragma omp parallel
     {
@@ -470,7 +482,7 @@ int oracle_forward_tokens_w8(const uint16_t* x, const float* logits,
                     const int e = ids[j];
                     if (!q13_e[e] || !s13_e[e] || !q2_e[e] || !s2_e[e]) { missing = 1; break; }
                     expert_ffn_row_w8(x + (size_t)t * H, q13_e[e], s13_e[e], q2_e[e], s2_e[e], H,
-                                      I, act, yk + (size_t)j * H);
+                                      I, dec, act, yk + (size_t)j * H);
                 }
                 if (missing) {
 #pragma omp atomic write
