@@ -84,7 +84,8 @@ typedef void* moe_stream_t;   /* cudaStream_t */
 size_t moe_workspace_size(moe_shape_t shape);
 
 /* route.  logits fp32 [T, E] -> topk_ids int32 [T, k], topk_weights fp32 [T, k]
- * (both ordered by selection rank).  Needs no workspace. */
+ * (both ordered by selection rank).  Needs no workspace, so it takes none: each
+ * token's selection and softmax stay in registers and shared memory. */
 moe_status_t moe_route(const float* logits, moe_shape_t shape, int32_t* topk_ids,
                        float* topk_weights, moe_stream_t stream);
 
@@ -121,7 +122,13 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
  * multi-launch path's (MOE_DISABLE_FUSED=1 in the environment selects that
  * path) bit for bit where that path leaves w13 unsplit (H < 512), and up to
  * bf16 rounding of the differently ordered sum otherwise.  Either way every
- * wait is bounded (2 s; then moe_device_status reports MOE_ERR_DEVICE_TIMEOUT). */
+ * wait is bounded (2 s; then moe_device_status reports MOE_ERR_DEVICE_TIMEOUT).
+ * Co-residency: that one launch has one CTA per SM, and its CTAs wait for each
+ * other's rows, so it assumes all of its CTAs run at once.  Kernels on other
+ * streams that hold SMs while it starts delay some of its CTAs; the call stays
+ * correct as long as they get an SM within the 2 s bound, and otherwise its
+ * output is unspecified and moe_device_status reports MOE_ERR_DEVICE_TIMEOUT
+ * (it never hangs).  Give it the device to itself for guaranteed progress. */
 moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
                          const moe_bf16_t* w2, moe_shape_t shape, moe_bf16_t* out,
                          int32_t* topk_ids, float* topk_weights, int32_t* expert_offsets,
@@ -158,9 +165,12 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
  * The first call on each device looks up the array's device address for that
  * device (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture.
- * Every call shares the one array: calls whose GPU work can overlap (on other
- * streams or host threads, same device) race and may return wrong results;
- * order them on one stream. */
+ * Every call shares the one array, which holds the per-chunk expert counts and
+ * also the per-expert tile list and its count: every call rewrites all of them,
+ * so after a later call only the caller's own output buffers still hold this
+ * call's results.  Calls whose GPU work can overlap (on other streams or host
+ * threads, same device) race and may return wrong results; order them on one
+ * stream. */
 #define MOE_PERMUTE_NOALLOC_MAX_ROWS (1 << 20)
 #define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (2097152 + 32768 + 256)
 moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
@@ -174,8 +184,9 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
  * weight (e, r, c) = e4m3(code) * scale(e, r).  Everything else -- arguments,
  * outputs, workspace (moe_workspace_size), routing, roundings, error reporting
  * -- is moe_forward's.  The weights stream at one byte each and are widened to
- * bf16 exactly in shared memory, so the tensor-core products are those of the
- * bf16 path; each weight row's scale multiplies its fp32 accumulator row.  Runs
+ * bf16 exactly on chip (into tensor memory, the MMA's A operand), so the
+ * tensor-core products are those of the bf16 path; each weight row's scale
+ * multiplies its fp32 accumulator row.  Runs
  * only as the one-launch FFN (moe_forward_w8_supported; 2 kernels):
  * MOE_ERR_UNSUPPORTED_SHAPE otherwise, whatever MOE_DISABLE_FUSED says.  Codes
  * 0x7F / 0xFF (NaN) propagate as NaN.  All pointers 16-byte aligned. */

@@ -208,16 +208,7 @@ __global__ void __launch_bounds__(256)
 template <typename Kern, typename... Args>
 cudaError_t launch_1d(Kern kern, long n, cudaStream_t st, Args... args)
 {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((n + 255) / 256));
-    cfg.blockDim = dim3(256);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    return launch_pdl(kern, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, args...);
 }
 
 }  // namespace
@@ -244,18 +235,10 @@ cudaError_t launch_combine_partials(const float* partials, const int32_t* splits
 {
     if (T == 0) return cudaSuccess;
     const int H4 = H / 4;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)T, (unsigned)((H4 + 63) / 64));
-    cfg.blockDim = dim3((unsigned)(64 * k));
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, combine_partials_kernel, reinterpret_cast<const float4*>(partials),
-                              splits, static_cast<const uint2*>(y), weights, T, k, H4,
-                              static_cast<uint2*>(out));
+    return launch_pdl(combine_partials_kernel, dim3((unsigned)T, (unsigned)((H4 + 63) / 64)),
+                      dim3((unsigned)(64 * k)), 0, st, reinterpret_cast<const float4*>(partials),
+                      splits, static_cast<const uint2*>(y), weights, T, k, H4,
+                      static_cast<uint2*>(out));
 }
 
 cudaError_t launch_swiglu_finalize(const float* partials, const int32_t* splits, int R, int I,

@@ -1002,17 +1002,8 @@ cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const
     auto kern = fused_ffn_kernel<NT, W8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(W8 ? W8Cfg<NT>::kThreads : kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, t13, t2, ta, a);
+    return launch_pdl(kern, dim3(grid), dim3(W8 ? W8Cfg<NT>::kThreads : kThreads), smem, st, t13,
+                      t2, ta, a);
 }
 
 }  // namespace

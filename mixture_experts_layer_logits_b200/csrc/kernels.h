@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "moe.h"
+
 namespace moe {
 
 // Value a kernel stores in the workspace's error word when it gives up on a
@@ -46,8 +48,33 @@ struct PermuteAux {
 // Records the cudaError_t that moe_last_cuda_error() reports on this host thread.
 void set_last_cuda_error(int err);
 
+// The shape rules of moe_route / moe_permute (1 <= E <= 1024, 1 <= k <= min(E, 16),
+// T >= 1, T*k <= 2^30); H and I are not looked at.
+bool routing_shape_ok(const moe_shape_t& s);
+
 // Launch helper: programmatic dependent launch unless MOE_DISABLE_PDL=1.
 bool pdl_enabled();
+
+// Launches kern<<<grid, block, smem, st>>>(args...) with programmatic dependent
+// launch allowed (unless MOE_DISABLE_PDL=1): the kernel may start while its
+// predecessor on `st` is finishing, and waits for it with griddepcontrol.wait
+// before reading that predecessor's results.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* weights,
                          cudaStream_t st);

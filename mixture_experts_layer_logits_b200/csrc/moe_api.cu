@@ -38,6 +38,13 @@ thread_local int g_last_cuda_error = 0;
 
 void set_last_cuda_error(int err) { g_last_cuda_error = err; }
 
+bool routing_shape_ok(const moe_shape_t& s)
+{
+    if (s.T < 1 || s.E < 1 || s.E > 1024 || s.top_k < 1 || s.top_k > 16 || s.top_k > s.E)
+        return false;
+    return (long long)s.T * s.top_k <= (1LL << 30);
+}
+
 namespace {
 
 // Plans and workspaces are sized for the B200's SM count; the launch grid uses
@@ -48,13 +55,6 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-bool routing_shape_ok(const moe_shape_t& s)
-{
-    if (s.T < 1 || s.E < 1 || s.E > 1024 || s.top_k < 1 || s.top_k > 16 || s.top_k > s.E)
-        return false;
-    return (long long)s.T * s.top_k <= (1LL << 30);
-}
 
 bool ffn_shape_ok(const moe_shape_t& s)
 {

@@ -60,8 +60,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t
 {
     using namespace moe;
     if (!topk_ids || !expert_offsets || !permuted_rows) return MOE_ERR_INVALID_ARG;
-    if (s.T < 1 || s.E < 1 || s.E > 1024 || s.top_k < 1 || s.top_k > 16 || s.top_k > s.E)
-        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!routing_shape_ok(s)) return MOE_ERR_UNSUPPORTED_SHAPE;  // moe_permute's rules
     const long long R = (long long)s.T * s.top_k;
     if (R > MOE_PERMUTE_NOALLOC_MAX_ROWS) return MOE_ERR_UNSUPPORTED_SHAPE;
     if ((reinterpret_cast<uintptr_t>(topk_ids) | reinterpret_cast<uintptr_t>(expert_offsets) |

@@ -580,17 +580,7 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int32_t* __rest
 template <typename Kern, typename... Args>
 cudaError_t launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args)
 {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    return launch_pdl(kern, grid, block, smem, st, args...);
 }
 
 int values_per_lane(int E)

@@ -50,6 +50,29 @@ def assert_routing_equal(ids, w, ref_ids, ref_w):
     assert dw <= WEIGHT_ATOL, f"topk_weights differ by {dw:.3e}"
 
 
+def library_tile_rows(T):
+    """Token rows per tile of the grouped GEMMs for T tokens: the smallest power of
+    two >= T, between 16 and 256 (each expert's segment is cut into tiles of this
+    many rows, the last one ragged)."""
+    nt = 16
+    while nt < 256 and nt < T:
+        nt *= 2
+    return nt
+
+
+def tile_boundary_tokens(expert_offsets, permuted_rows, k, nt):
+    """Tokens whose expanded rows are the first or the last row of some nt-row tile
+    of some expert's segment: every tile of the grouped GEMMs, its ragged tail
+    and every segment boundary then holds at least one checked row."""
+    pos = set()
+    for e in range(len(expert_offsets) - 1):
+        a, b = int(expert_offsets[e]), int(expert_offsets[e + 1])
+        for s in range(a, b, nt):
+            pos.add(s)
+            pos.add(min(s + nt, b) - 1)
+    return sorted({int(permuted_rows[p]) // k for p in pos})
+
+
 def expert_weights_for(tokens, ref_ids, w13, w2):
     """Host copies of only the experts the listed tokens select (per-expert lists)."""
     E = w13.shape[0]

@@ -3,10 +3,15 @@ include/moe.h declares, and rejects bad arguments before touching a device.
 
 Nothing here launches work: every call is made with arguments that host-side
 validation rejects, or is a pure host function (workspace sizing, status text).
+The calls pass made-up "device" addresses, so the tests run in a child process
+that sees no GPU (CUDA_VISIBLE_DEVICES empty): should host validation ever let
+one through, the call fails with a CUDA error instead of reaching a real device.
 """
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -14,6 +19,7 @@ import mixture_experts_layer_logits_b200 as moe
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe.h")
+NO_DEVICE = os.environ.get("CUDA_VISIBLE_DEVICES") == ""
 
 # a fake, 16-byte aligned "device" address: validation never dereferences it
 A = ctypes.c_void_p(0x7f0000001000)
@@ -21,8 +27,20 @@ MIS = ctypes.c_void_p(0x7f0000001004)
 NUL = None
 
 
+@pytest.mark.skipif(NO_DEVICE, reason="this is the child process")
+def test_boundary_checks_in_a_process_without_a_device():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "-m", "not gpu", os.path.abspath(__file__)],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout and " failed" not in r.stdout, r.stdout[-2000:]
+
+
 @pytest.fixture(scope="module")
 def lib():
+    if not NO_DEVICE:
+        pytest.skip("runs in the child process without a device")
     from mixture_experts_layer_logits_b200 import build
 
     build.build()
@@ -224,3 +242,15 @@ def test_selftest_wait_timeout_validation(lib):
     assert f(A, 64, 2000001, NUL) == moe.MOE_ERR_INVALID_ARG
     assert f(MIS, 64, 1000, NUL) == moe.MOE_ERR_MISALIGNED
     assert f(A, 4, 1000, NUL) == moe.MOE_ERR_WORKSPACE_TOO_SMALL   # needs the error word + a flag
+
+
+def test_permute_noalloc_rejects_sizes_beyond_its_scratch(lib):
+    fn = lib.moe_permute_noalloc
+    fn.argtypes = [ctypes.c_void_p, moe.Shape, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    k = 8
+    T = (1 << 20) // k + 1                       # one row past the scratch's limit
+    assert fn(A, moe.Shape(T, 64, k, 0, 0), A, A, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert fn(NUL, moe.Shape(8, 64, k, 0, 0), A, A, None) == moe.MOE_ERR_INVALID_ARG
+    assert fn(A, moe.Shape(8, 2000, k, 0, 0), A, A, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert fn(A, moe.Shape(8, 64, k, 0, 0), MIS, A, None) == moe.MOE_ERR_MISALIGNED

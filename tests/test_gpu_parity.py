@@ -16,7 +16,7 @@ import mixture_experts_layer_logits_b200 as moe
 from mixture_experts_layer_logits_b200 import workloads as wl
 
 from parity import (assert_out_close, assert_routing_equal, expert_weights_for, host_bits,
-                    host_f32)
+                    host_f32, library_tile_rows, tile_boundary_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -150,33 +150,57 @@ def test_forward_full_configs(name):
     check_full(w, inputs(w))
 
 
-def sampled_check(w, d, n_tokens, seed=0):
+def check_tokens(w, d, pick):
+    """Routing and permutation in full; the layer output of the tokens that
+    pick(ref_offsets, ref_rows) lists against the oracle's forward_tokens (a
+    token's output depends only on its own row), with host copies of only the
+    experts those tokens select."""
     out, ids, wts, off, rows = run_forward(w, d)
     ref_ids, ref_w = oracle.route(host_f32(d["logits"]), w.k)
     assert_routing_equal(ids, wts, ref_ids, ref_w)
     ref_off, ref_rows = oracle.permute(ref_ids, w.E)
     np.testing.assert_array_equal(off.cpu().numpy(), ref_off)
     np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)
-    rng = np.random.default_rng(seed)
-    toks = sorted(set([0, w.T - 1] + rng.choice(w.T, size=n_tokens, replace=False).tolist()))
+    toks = pick(ref_off, ref_rows)
     w13s, w2s = expert_weights_for(toks, ref_ids, d["w13"], d["w2"])
     ref = oracle.forward_tokens(host_bits(d["x"]), host_f32(d["logits"]), w13s, w2s, w.k, toks,
                                 w.I)
-    return assert_out_close(out[toks], ref, what=f"out[{len(toks)} sampled tokens]")
+    return assert_out_close(out[toks], ref, what=f"out[{len(toks)} of {w.T} tokens]")
 
 
-def test_forward_skewed_decode_sampled():
+def test_forward_skewed_decode_all_tokens():
+    """The skewed-decode layer (T=64, E=256, k=8, H=7168, I=2048, Zipf-hot experts)
+    against the oracle on every token."""
     w = wl.WORKLOADS["skewed_decode"]
     d = inputs(w)
-    sampled_check(w, d, n_tokens=10)
+    check_tokens(w, d, lambda off, rows: list(range(w.T)))
     del d
     torch.cuda.empty_cache()
 
 
-def test_forward_prefill_sampled():
+def test_forward_prefill_every_tile():
+    """The prefill layer (T=8192, E=128, k=8, H=4096, I=1536) against the oracle on
+    every token whose row is the first or the last row of a 256-row tile of an
+    expert's segment: every (expert, tile) of both grouped GEMMs, every ragged
+    tail and every segment boundary holds a checked row, and the other rows of
+    those tokens land anywhere inside other tiles."""
     w = wl.WORKLOADS["prefill"]
     d = inputs(w)
-    sampled_check(w, d, n_tokens=8)
+    nt = library_tile_rows(w.T)
+    assert nt == 256
+
+    def pick(off, rows):
+        toks = tile_boundary_tokens(off, rows, w.k, nt)
+        checked = np.zeros(w.T * w.k, bool)
+        for t in toks:
+            checked[t * w.k:(t + 1) * w.k] = True
+        # every tile of every expert holds at least one checked row
+        for e in range(w.E):
+            for s in range(int(off[e]), int(off[e + 1]), nt):
+                assert checked[rows[s:min(s + nt, int(off[e + 1]))]].any(), (e, s)
+        return toks
+
+    check_tokens(w, d, pick)
     del d
     torch.cuda.empty_cache()
 
@@ -311,10 +335,13 @@ def test_fused_launch_against_multi_launch_and_oracle(tmp_path):
             assert torch.equal(out.cpu(), multi), name
         else:
             assert_out_close(out, multi.float().numpy().astype(np.float64), what=f"{name} vs multi-launch")
-        # the one-launch result against the oracle, on sampled tokens
+        # the one-launch result against the oracle
         ref_ids, ref_w = oracle.route(host_f32(d["logits"]), w.k)
         assert_routing_equal(ids, wts, ref_ids, ref_w)
-        toks = sorted(set([0, w.T // 2, w.T - 1]))
+        # every token where the oracle is cheap; skewed decode is checked on every
+        # token through the same one-launch path by its own test
+        small = w.T * w.k * 3 * w.H * w.I <= 4e9
+        toks = list(range(w.T)) if small else sorted(set([0, w.T // 2, w.T - 1]))
         w13s, w2s = expert_weights_for(toks, ref_ids, d["w13"], d["w2"])
         want = oracle.forward_tokens(host_bits(d["x"]), host_f32(d["logits"]), w13s, w2s, w.k,
                                      toks, w.I)

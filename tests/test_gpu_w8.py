@@ -90,9 +90,9 @@ def test_forward_w8_matches_oracle(name, spec):
     assert_out_close(out, ref["out"], what=f"{name} out")
 
 
-def test_forward_w8_skewed_decode_sampled():
-    """The full skewed-decode shape (T=64, E=256, k=8, H=7168, I=2048) on sampled
-    tokens: the oracle gets only the experts those tokens select."""
+def test_forward_w8_skewed_decode_all_tokens():
+    """The full skewed-decode shape (T=64, E=256, k=8, H=7168, I=2048) on every
+    token: the oracle gets only the experts the tokens select."""
     w = wl.WORKLOADS["skewed_decode"]
     d = w8_inputs(w, seed=0)
     out, ids, wts, off, rows = run_w8(w, d)
@@ -101,15 +101,14 @@ def test_forward_w8_skewed_decode_sampled():
     ref_off, ref_rows = oracle.permute(ref_ids, w.E)
     np.testing.assert_array_equal(off.cpu().numpy(), ref_off)
     np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)
-    rng = np.random.default_rng(0)
-    toks = sorted(set([0, w.T - 1] + rng.choice(w.T, size=8, replace=False).tolist()))
+    toks = list(range(w.T))
     experts = [None] * w.E
-    for e in sorted(set(ref_ids[toks].reshape(-1).tolist())):
+    for e in sorted(set(ref_ids.reshape(-1).tolist())):
         experts[e] = (host_u8(d["q13"][e]), host_f32(d["s13"][e]), host_u8(d["q2"][e]),
                       host_f32(d["s2"][e]))
     want = oracle.forward_tokens_w8(host_bits(d["x"]), host_f32(d["logits"]), experts, w.k, toks,
                                     w.I)
-    assert_out_close(out[toks], want, what=f"out[{len(toks)} sampled tokens]")
+    assert_out_close(out, want, what="out (all 64 tokens)")
     del d
     torch.cuda.empty_cache()
 

@@ -5,7 +5,9 @@ Checked through the C ABI against moe_permute, the entry point that takes a
 workspace: the results must be bit-identical, on two calls in a row (the second
 call must not be disturbed by what the first left in the shared array).  This
 file is collected last so that a run stopping at the first failure has already
-run every other test; it also passes on its own in a fresh process.
+run every other test; it also passes on its own in a fresh process.  (Its
+rejection of sizes beyond the scratch is checked on the host, without a device,
+in test_boundary.py.)
 """
 import ctypes
 
@@ -55,8 +57,10 @@ def _with_workspace(ids, E):
     return moe.moe_permute(ids, E, ws=ws)
 
 
+# the last case fills the scratch to its limit: T*k = 2^20 rows, 512 chunks of
+# counts at E = 1024, right below the tile list
 CASES = [(8, 128, 8, False), (16384, 1024, 8, False), (5000, 37, 3, True), (512, 8, 8, False),
-         (70000, 256, 8, True)]
+         (70000, 256, 8, True), (MAX_ROWS // 8, 1024, 8, True)]
 
 
 @pytest.mark.gpu
@@ -73,14 +77,3 @@ def test_noalloc_matches_workspace_permute_on_consecutive_calls():
         for got, want in ((got_a, want_a), (got_b, want_b)):
             np.testing.assert_array_equal(got[0].cpu().numpy(), want[0].cpu().numpy())
             np.testing.assert_array_equal(got[1].cpu().numpy(), want[1].cpu().numpy())
-
-
-def test_noalloc_rejects_sizes_beyond_its_scratch():
-    lib = _lib()
-    fake = ctypes.c_void_p(0x7f0000001000)   # never dereferenced: rejected on the host
-    k = 8
-    T = MAX_ROWS // k + 1
-    rc = lib.moe_permute_noalloc(fake, moe.Shape(T, 64, k, 0, 0), fake, fake, None)
-    assert rc == moe.MOE_ERR_UNSUPPORTED_SHAPE
-    assert lib.moe_permute_noalloc(None, moe.Shape(8, 64, k, 0, 0), fake, fake,
-                                   None) == moe.MOE_ERR_INVALID_ARG
