@@ -103,11 +103,14 @@ __device__ __forceinline__ int split_count(int units, int s_max, int num_kt, int
 }
 
 // silu(g) * u = g * u / (1 + e^-g).  The result is rounded to bf16 (8-bit
-// significand), so the fast exponential and reciprocal (a few ulp of fp32) are
-// far inside that rounding; for g -> -inf the reciprocal of inf is 0.
+// significand), so the fast exponential and the approximate reciprocal (one
+// MUFU instruction each, a few ulp of fp32) are far inside that rounding; when
+// e^-g overflows, the reciprocal of inf is 0.
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
-    return g * __frcp_rn(1.0f + __expf(-g)) * u;
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + __expf(-g)));
+    return g * r * u;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int n)

@@ -15,25 +15,32 @@
 // memory (fp32); MODE 0 keeps a gate and an up accumulator of equal shape so the
 // epilogue thread that owns feature f holds both halves of its SwiGLU pair.
 //
-// Warp roles (512 threads):
+// Warp roles:
 //   warp 0      TMA producer: weight tiles [128 x 64] (and, MODE 1, the act tile
 //               [NT x 64]) with the 128-byte swizzle into a STAGES-deep ring.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
-//   warps 2-7   MODE 0 activation gather, in G = min(6, stages) groups of 6 / G
-//               warps; group g owns every stage whose sequence number is g mod G.
-//               It issues 16-byte cp.async copies of the x rows selected by
-//               permuted_rows[p] / k straight into the swizzled B tile (no permuted
-//               copy of x exists), waits for them, then fence.proxy.async and one
-//               mbarrier arrival per warp -- the writer-side proxy fence and barrier
-//               the FlashInfer PR #7368 page ("2. Hopper") requires before an async
-//               proxy reads generic-proxy stores.  The weight TMA of a stage is issued
-//               independently of its gather, so the two overlap (the BF16 ordering of
-//               the same section).  At most one group per stage keeps every waiter
-//               within one mbarrier phase of its slot.  Idle in MODE 1.
-//   warps 8-15  epilogue, two groups of four: tcgen05.ld of the accumulator
-//               (warp w reads TMEM lanes 32*(w%4) ..), group h owning the token
-//               columns [h*NT/2, (h+1)*NT/2); SwiGLU / bf16 rounding / scatter, or
-//               split-K partials.
+//   MODE 0: warps 2-5 activation gather.  Every gather thread copies part of
+//               every stage: 16-byte cp.async copies of the x rows selected by
+//               permuted_rows[p] / k straight into the swizzled B tile (no
+//               permuted copy of x exists).  Each thread's copies arrive on the
+//               stage's mbarrier when they land (cp.async.mbarrier.arrive), so no
+//               gather thread waits for its own copies; the MMA thread issues the
+//               async-proxy fence after that barrier and before its MMAs read the
+//               tile -- the proxy fence plus barrier that the FlashInfer PR #7368
+//               page ("2. Hopper") requires before an async proxy reads
+//               generic-proxy writes.  The weight TMA of a stage is issued
+//               independently of its gather, so the two overlap (the BF16 ordering
+//               of the same section).
+//   epilogue    MODE 0: warps 6-13, two groups of four; MODE 1: warps 2-17, four
+//               groups of four (two when NT < 64).  Warp w reads TMEM lanes
+//               32*(w%4) ..; group g owns a contiguous range of token columns.  It
+//               drains its columns into registers as packed bf16 (MODE 0: SwiGLU
+//               applied), hands them back to the MMA thread at once, and only then
+//               stages and stores the rows, so the stores overlap the next unit's
+//               main loop.  MODE 1 hands back its two 128-row output blocks one at
+//               a time, and the MMA thread starts the next unit on the first block
+//               while the second is still being drained.  Split-K units write fp32
+//               partials instead.
 //
 // Split-K: when there are too few (tile, feature block) units to fill the GPU
 // (decode), each unit's K range is cut into S slices (S chosen on the device
@@ -80,35 +87,107 @@ struct FfnArgs {
     int weights_evict_first;  // weights are streamed once (few tokens per expert)
 };
 
-__device__ __forceinline__ void flag_error(const FfnArgs& a, Aux* aux)
+// Thread roles of the grouped GEMM:
+//   warp 0              TMA producer
+//   warp 1              TMEM allocator and MMA issuer
+//   MODE 0 (14 warps):  warps 2-5 activation gather; warps 6-13 epilogue (2 groups of 4)
+//   MODE 1 (18 warps):  warps 2-17 epilogue (4 groups of 4; 2 groups, warps 2-9, when
+//                       NT < 64)
+constexpr int kGGatherWarps = 4;
+constexpr int kGGatherThreads = kGGatherWarps * 32;
+
+template <int MODE, int NT>
+struct GCfg {
+    // MODE 0: 2 + 4 gather + 8 epilogue warps; MODE 1: 2 + 16 epilogue warps
+    static constexpr int kThreads = MODE == 0 ? 448 : 576;
+    static constexpr int kNA = 2;                                  // A tiles per stage
+    static constexpr int kBTileBytes = NT * kBK * 2;
+    static constexpr int kStageBytes = kNA * kATileBytes + kBTileBytes;
+    static constexpr int kMaxSmem = 232448;                        // 227 KB per CTA
+    // epilogue groups: 4 warps each (one per TMEM lane quarter), each group owning
+    // kGroupCols consecutive token columns of the accumulator
+    static constexpr int kGroups = (MODE == 1 && NT >= 64) ? 4 : 2;
+    static constexpr int kEpiWarp0 = MODE == 0 ? 2 + kGGatherWarps : 2;
+    static constexpr int kEpiWarps = 4 * kGroups;
+    static constexpr int kGroupCols = NT / kGroups;
+    static constexpr int kRows = 8;                                // token rows per staging chunk
+    static constexpr int kRowBytes = 256;                          // one staged row segment
+    static constexpr int kStagingBytes = kGroups * 2 * kRows * kRowBytes;
+    // rows of the B tile one gather thread copies per stage (8 16-byte chunks a row)
+    static constexpr int kGIters = (NT * 8 + kGGatherThreads - 1) / kGGatherThreads;
+    static constexpr int kAuxBytes = 1024;
+    static constexpr int kStagesRaw = (kMaxSmem - 1024 - kAuxBytes - kStagingBytes) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kAccCols = 2 * NT;                        // per accumulator buffer
+    static constexpr int kNBufRaw = 512 / kAccCols;
+    static constexpr int kNBuf = kNBufRaw > 8 ? 8 : kNBufRaw;
+    static constexpr int kUsedCols = kAccCols * kNBuf;
+    static constexpr int kTmemCols = kUsedCols <= 32 ? 32 : kUsedCols <= 64 ? 64
+                                   : kUsedCols <= 128 ? 128 : kUsedCols <= 256 ? 256 : 512;
+    static constexpr uint32_t kTxBytes = kNA * kATileBytes + (MODE == 1 ? kBTileBytes : 0);
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kStagingBytes + kAuxBytes;
+    // token columns per tcgen05.ld in the split-K epilogue (within the group's columns)
+    static constexpr int kLdCols = kGroupCols >= 16 ? 16 : 8;
+    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N tile");
+    static_assert(kGroupCols % 8 == 0 && kGroupCols % kRows == 0, "epilogue column split");
+    static_assert(kStages >= 2, "pipeline depth");
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kSmemBytes <= kMaxSmem, "shared memory");
+    static_assert(kEpiWarp0 + kEpiWarps <= kThreads / 32, "warp roles");
+};
+
+// Barriers of one CTA.  tempty[b] frees accumulator buffer b (MODE 1: its first
+// 128-row block's columns only) and tempty2[b] (MODE 1) its second block's, so
+// the next unit's MMAs into the first block can start while the epilogue still
+// drains the second.
+struct GAux {
+    uint64_t full[16];
+    uint64_t empty[16];
+    uint64_t tfull[8];
+    uint64_t tempty[8];
+    uint64_t tempty2[8];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void flag_error(const FfnArgs& a, GAux* aux)
 {
     atomicExch(a.err, kDeviceErrorMagic);
     aux->abort = 1;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 template <int MODE, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_act, const FfnArgs a)
 {
-    using C = Cfg<MODE, NT>;
+    using C = GCfg<MODE, NT>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t* staging = ring + C::kStages * C::kStageBytes;
-    Aux* aux = reinterpret_cast<Aux*>(staging + C::kStagingBytes);
-    int* tok_off = reinterpret_cast<int*>(aux + 1);
+    GAux* aux = reinterpret_cast<GAux*>(staging + C::kStagingBytes);
+    static_assert(sizeof(GAux) <= C::kAuxBytes, "aux area");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&aux->full[s], MODE == 0 ? 1 + C::kW : 1);
+            // MODE 0: the producer's expect_tx plus one arrival per gather warp
+            mbar_init(&aux->full[s], MODE == 0 ? 1 + kGGatherWarps : 1);
             mbar_init(&aux->empty[s], 1);
         }
         for (int b = 0; b < C::kNBuf; ++b) {
             mbar_init(&aux->tfull[b], 1);
-            mbar_init(&aux->tempty[b], 8);
+            mbar_init(&aux->tempty[b], C::kEpiWarps);
+            mbar_init(&aux->tempty2[b], C::kEpiWarps);
         }
         mbar_init(&aux->drain, 1);
         aux->abort = 0;
@@ -240,11 +319,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Per K tile: two MMAs (gate and up blocks, or two 128-row w2 blocks) into
+        // accumulators d0 and d0 + NT.  MODE 1 starts a unit with the first
+        // block's MMAs of up to kStages K tiles, which need only tempty[b], and
+        // waits for tempty2[b] (the epilogue still draining the previous unit's
+        // second block) before the second block's.
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int lu = 0;
             bool ok = true;
+            auto wait_full = [&](int st_, uint32_t ph_) {
+                if (!mbar_wait(&aux->full[st_], ph_, abort_flag)) {
+                    flag_error(a, aux);
+                    return false;
+                }
+                // MODE 0: the B tile was written by cp.async (generic proxy); the
+                // tensor core reads it through the async proxy
+                if (MODE == 0) fence_proxy_async_smem();
+                tc_fence_after();
+                return true;
+            };
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++lu) {
                 int split, tile, fb;
                 decode(u, split, tile, fb);
@@ -260,23 +355,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n = (t.rows + 15) & ~15;
                 const uint32_t idesc = umma_idesc_bf16(kBM, n);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::kAccCols);
-                for (int kt = kt0; kt < kt1; ++kt) {
-                    if (!mbar_wait(&aux->full[stage], phase, abort_flag)) {
+                auto issue = [&](uint32_t d, int st_, int blk, bool first_kt) {
+                    const uint32_t sa = smem_u32(ring + st_ * C::kStageBytes);
+                    const uint32_t bt = sa + C::kNA * kATileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+                        umma_bf16(d, umma_desc_sw128(sa + blk * kATileBytes + kk * 32),
+                                  umma_desc_sw128(bt + kk * 32), idesc,
+                                  (!first_kt || kk > 0) ? 1u : 0u);
+                };
+                int kt = kt0;
+                if (MODE == 1) {
+                    // first block over the first n_pre K tiles, then the second block
+                    const int n_pre = min(C::kStages, kt1 - kt0);
+                    for (int i = 0; i < n_pre && ok; ++i) {
+                        const int st_ = (stage + i) % C::kStages;
+                        const uint32_t ph_ = phase ^ (uint32_t)((stage + i) / C::kStages);
+                        ok = wait_full(st_, ph_);
+                        if (ok) issue(d0, st_, 0, i == 0);
+                    }
+                    if (ok && !mbar_wait(&aux->tempty2[b], aphase ^ 1u, abort_flag)) {
                         flag_error(a, aux);
+                        ok = false;
+                    }
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int i = 0; i < n_pre; ++i) {
+                        issue(d0 + NT, stage, 1, i == 0);
+                        umma_commit(&aux->empty[stage]);  // frees the smem stage when read
+                        if (++stage == C::kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    kt += n_pre;
+                }
+                for (; kt < kt1; ++kt) {
+                    if (!wait_full(stage, phase)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t st = smem_u32(ring + stage * C::kStageBytes);
-                    const uint32_t bt = st + C::kNA * kATileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        const uint32_t acc = (kt > kt0 || kk > 0) ? 1u : 0u;
-                        const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
-                        umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
-                        umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
-                                  idesc, acc);
-                    }
+                    issue(d0, stage, 0, kt == kt0);
+                    issue(d0 + NT, stage, 1, kt == kt0);
                     umma_commit(&aux->empty[stage]);  // frees the smem stage when read
                     if (++stage == C::kStages) {
                         stage = 0;
@@ -290,72 +410,74 @@ __global__ void __launch_bounds__(kThreads, 1)
             volatile int never = 0;
             if (!mbar_wait(&aux->drain, 0, &never, 500000000ull)) atomicExch(a.err, kDeviceErrorMagic);
         }
-    } else if (warp < 2 + kGatherWarps) {
+    } else if (MODE == 0 && warp < 2 + kGGatherWarps) {
         // ------------------------------------------------------------ gather (MODE 0)
-        if (MODE == 0 && warp - 2 < C::kG * C::kW) {
-            constexpr int G = C::kG, W = C::kW;
-            const int g = (warp - 2) / W, wi = (warp - 2) % W;
-            int* my_off = tok_off + (warp - 2) * NT;
-            const uint64_t x_policy = l2_policy_evict_last();  // x rows are re-read per block
-            int q = 0;         // global stage sequence number (same as producer's)
-            int cur_tile = -1;
-            bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                int split, tile, fb;
-                decode(u, split, tile, fb);
-                const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
-                // first stage of this unit that this warp owns
-                int kt = kt0 + ((g - q % G) + G) % G;
-                const int q_unit0 = q;
-                q += kt1 - kt0;
-                if (kt >= kt1) continue;
+        // Every gather warp fills part of every stage: gather thread g copies the
+        // 16-byte chunks g, g + 128, ... of the tile's B rows (row = chunk / 8), so a
+        // warp instruction covers 4 whole 128-byte row segments.  Each thread's
+        // copies arrive on the stage's full barrier when they land
+        // (cp.async.mbarrier.arrive), then the warp arrives once: no thread waits
+        // for its own copies, and the barrier completes only when every copy and
+        // the weight TMA have landed.  The MMA thread fences the async proxy
+        // before reading the tile.
+        const int g = threadIdx.x - 64;  // 0 .. kGGatherThreads - 1
+        const uint64_t x_policy = l2_policy_evict_last();  // x rows are re-read per block
+        int off[C::kGIters];  // element offset of this thread's x row per iteration (-1: none)
+        int q = 0;            // global stage sequence number (same as the producer's)
+        int cur_tile = -1;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int split, tile, fb;
+            decode(u, split, tile, fb);
+            const int kt0 = split * kt_per_split, kt1 = min(a.num_kt, kt0 + kt_per_split);
+            if (tile != cur_tile) {
                 const Tile t = load_tile(a.tiles + tile);
-                if (tile != cur_tile) {
-                    __syncwarp();  // earlier copies' addresses are all issued
-                    for (int j = lane; j < t.rows; j += 32)
-                        my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
-                    __syncwarp();
-                    cur_tile = tile;
+#pragma unroll
+                for (int i = 0; i < C::kGIters; ++i) {
+                    const int j = (g + i * kGGatherThreads) >> 3;
+                    off[i] = j < t.rows ? (a.permuted_rows[t.row_start + j] / a.k) * a.H + (g & 7) * 8
+                                        : -1;
                 }
-                const int chunks = t.rows * 8;
-                for (; kt < kt1; kt += G) {
-                    const int qq = q_unit0 + (kt - kt0);
-                    const int stage = qq % C::kStages;
-                    const uint32_t phase = (uint32_t)((qq / C::kStages) & 1);
-                    // warp-uniform decision, so no lane is left behind at __syncwarp
-                    if (!__all_sync(0xffffffffu, mbar_wait(&aux->empty[stage], phase ^ 1u,
-                                                           abort_flag))) {
-                        if (lane == 0) flag_error(a, aux);
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t bt =
-                        smem_u32(ring + stage * C::kStageBytes + C::kNA * kATileBytes);
-                    const __nv_bfloat16* src0 = a.x + kt * kBK;
-                    for (int c8 = lane + 32 * wi; c8 < chunks; c8 += 32 * W) {
-                        const int j = c8 >> 3, c = c8 & 7;
-                        cp_async_16_hint(bt + j * 128 + ((c ^ (j & 7)) << 4),
-                                         src0 + my_off[j] + c * 8, x_policy);
-                    }
-                    cp_async_commit();
-                    cp_async_wait<0>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&aux->full[stage]);
-                }
+                cur_tile = tile;
             }
-            cp_async_wait<0>();
+            for (int kt = kt0; kt < kt1; ++kt, ++q) {
+                const int stage = q % C::kStages;
+                const uint32_t phase = (uint32_t)((q / C::kStages) & 1);
+                // warp-uniform decision, so no lane is left behind at __syncwarp
+                if (!__all_sync(0xffffffffu, mbar_wait(&aux->empty[stage], phase ^ 1u,
+                                                       abort_flag))) {
+                    if (lane == 0) flag_error(a, aux);
+                    ok = false;
+                    break;
+                }
+                const uint32_t bt = smem_u32(ring + stage * C::kStageBytes + C::kNA * kATileBytes);
+                const __nv_bfloat16* src0 = a.x + kt * kBK;
+#pragma unroll
+                for (int i = 0; i < C::kGIters; ++i) {
+                    const int c8 = g + i * kGGatherThreads;
+                    const int j = c8 >> 3, c = c8 & 7;
+                    if (off[i] >= 0)
+                        cp_async_16_hint(bt + j * 128 + ((c ^ (j & 7)) << 4), src0 + off[i],
+                                         x_policy);
+                }
+                cp_async_mbar_arrive(&aux->full[stage]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aux->full[stage]);
+            }
         }
-    } else {
+        cp_async_commit();
+        cp_async_wait<0>();  // no copy is still in flight when the CTA exits
+    } else if (warp >= C::kEpiWarp0 && warp < C::kEpiWarp0 + C::kEpiWarps) {
         // ------------------------------------------------------------ epilogue
-        if (warp < kEpiWarp0) goto teardown;
         if (MODE == 1) pdl_wait();  // the outputs and partials the predecessor reads
-        const int grp = (warp - kEpiWarp0) >> 2;  // token-column half
-        const int q = warp & 3;                 // TMEM lane quarter
-        const int f_local = q * 32 + lane;      // feature inside the 128-row block
+        const int grp = (warp - C::kEpiWarp0) >> 2;  // token-column group
+        const int q = warp & 3;                      // TMEM lane quarter
+        const int f_local = q * 32 + lane;           // feature inside the 128-row block
+        const int gt = (warp - C::kEpiWarp0 - grp * 4) * 32 + lane;  // 0..127 in the group
         const int pcols = (MODE == 0) ? 2 * a.I : a.H;
         const int ocols = (MODE == 0) ? a.I : a.H;
-        int chunk = 0;  // staging chunks issued by this group (buffer parity)
+        uint8_t* gstage = staging + grp * 2 * (C::kRows * C::kRowBytes);
+        int chunk = 0;  // staging chunks written by this group (buffer parity)
         int lu = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++lu) {
             int split, tile, fb;
@@ -372,89 +494,114 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = (MODE == 0 ? fb * kBM : fb * 2 * kBM) + f_local;
             const bool f1_ok = MODE == 0 || f + kBM < a.H;
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols);
-            const int jbeg = grp * (NT / 2), jend = min(t.rows, (grp + 1) * (NT / 2));
+            const int jbeg = grp * C::kGroupCols;
+            const int jend = min(t.rows, jbeg + C::kGroupCols);
             if (S == 1) {
-                // Stage 8 token rows at a time in shared memory ([row][256 outputs] bf16),
-                // then the group's 128 threads copy them out with 16-byte loads and
-                // stores, each output row written whole and coalesced (256 B of act in
-                // MODE 0, up to 512 B of y in MODE 1).  Two buffers per group: one
-                // barrier per chunk separates a buffer's readers from its next writers.
-                const int row_bytes = MODE == 0 ? 2 * kBM : ((fb * 2 + 1) * kBM < a.H ? 4 * kBM : 2 * kBM);
-                const int vec_per_row = row_bytes / 16;
-                for (int j0 = jbeg; j0 < jend; j0 += kStageRows) {
-                    uint32_t g[8], v[8];
-                    tmem_ld8(tacc + j0, g);
-                    tmem_ld8(tacc + NT + j0, v);
-                    tmem_ld_wait();
-                    if (j0 + kStageRows >= jend) {  // accumulator drained: let the MMA go on
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&aux->tempty[b]);
-                    }
-                    uint8_t* buf = staging + (grp * 2 + (chunk & 1)) * (kStageRows * kStageRowBytes);
+                // For each output block (MODE 0: act; MODE 1: the two 128-row w2
+                // blocks in turn):
+                // 1. drain this group's accumulator columns into registers as packed
+                //    bf16 (MODE 0: act = silu(gate) * up), then hand the columns back
+                //    to the MMA thread at once, so the next unit's main loop overlaps
+                //    the stores below;
+                // 2. stage kRows token rows at a time in shared memory (one 256-byte
+                //    row segment each) and copy them out with 16-byte loads and
+                //    stores, each row segment written whole.  Two buffers per group:
+                //    one barrier per chunk separates a buffer's readers from its next
+                //    writers.
+                constexpr int kPk = C::kGroupCols / 2;
+                constexpr int kBlocks = MODE == 0 ? 1 : 2;
 #pragma unroll
-                    for (int jj = 0; jj < kStageRows; ++jj) {
-                        __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(buf + jj * kStageRowBytes);
-                        if (MODE == 0) {
-                            row[f_local] = __float2bfloat16_rn(
-                                silu_mul(__uint_as_float(g[jj]), __uint_as_float(v[jj])));
-                        } else {
-                            row[f_local] = __float2bfloat16_rn(__uint_as_float(g[jj]));
-                            row[kBM + f_local] = __float2bfloat16_rn(__uint_as_float(v[jj]));
+                for (int h = 0; h < kBlocks; ++h) {
+                    uint32_t pk[kPk];
+#pragma unroll
+                    for (int c = 0; c < C::kGroupCols; c += 8) {
+                        if (jbeg + c < jend) {  // warp-uniform
+                            uint32_t gv[8];
+                            tmem_ld8(tacc + h * NT + jbeg + c, gv);
+                            if (MODE == 0) {
+                                uint32_t vv[8];
+                                tmem_ld8(tacc + NT + jbeg + c, vv);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int i = 0; i < 8; i += 2)
+                                    pk[(c + i) / 2] = pack_bf16x2(
+                                        silu_mul(__uint_as_float(gv[i]), __uint_as_float(vv[i])),
+                                        silu_mul(__uint_as_float(gv[i + 1]),
+                                                 __uint_as_float(vv[i + 1])));
+                            } else {
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int i = 0; i < 8; i += 2)
+                                    pk[(c + i) / 2] = pack_bf16x2(__uint_as_float(gv[i]),
+                                                                  __uint_as_float(gv[i + 1]));
+                            }
                         }
                     }
-                    named_bar_sync(1 + grp, 128);  // staged; the other buffer is free again
-                    const int n = min(kStageRows, jend - j0);
-                    const int gt = (warp & 3) * 32 + lane;  // 0..127 within the group
-                    for (int i = gt; i < n * vec_per_row; i += 128) {
-                        const int jj = i / vec_per_row, c = i % vec_per_row;
-                        const int p = t.row_start + j0 + jj;
-                        const uint4 val = *reinterpret_cast<const uint4*>(buf + jj * kStageRowBytes + c * 16);
-                        __nv_bfloat16* dst = MODE == 0
-                            ? a.out + (size_t)p * ocols + fb * kBM
-                            : a.out + (size_t)a.permuted_rows[p] * ocols + fb * 2 * kBM;
-                        *reinterpret_cast<uint4*>(dst + c * 8) = val;
-                    }
-                    ++chunk;
-                }
-                if (jbeg >= jend) {  // this group had no columns of the unit
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&aux->tempty[b]);
+                    if (lane == 0) mbar_arrive(h == 0 ? &aux->tempty[b] : &aux->tempty2[b]);
+                    // MODE 1: the second block of the last pair may lie past H
+                    if (h == 1 && !f1_ok) continue;
+                    // one 16-byte vector per group thread: kRows rows of 16 vectors
+                    const int jj = gt >> 4, cc = gt & 15;
+                    const int col0 = MODE == 0 ? fb * kBM : fb * 2 * kBM + h * kBM;
+#pragma unroll
+                    for (int c = 0; c < C::kGroupCols; c += C::kRows) {
+                        if (jbeg + c < jend) {  // group-uniform
+                            uint8_t* buf = gstage + (chunk & 1) * (C::kRows * C::kRowBytes);
+#pragma unroll
+                            for (int r = 0; r < C::kRows; ++r) {
+                                const uint32_t w = pk[(c + r) / 2];
+                                reinterpret_cast<uint16_t*>(buf + r * C::kRowBytes)[f_local] =
+                                    (uint16_t)(((c + r) & 1) ? (w >> 16) : (w & 0xFFFFu));
+                            }
+                            named_bar_sync(1 + grp, 128);  // staged; the other buffer is free again
+                            if (jj < jend - (jbeg + c)) {
+                                const int p = t.row_start + jbeg + c + jj;
+                                const uint4 val = *reinterpret_cast<const uint4*>(
+                                    buf + jj * C::kRowBytes + cc * 16);
+                                const size_t row = MODE == 0 ? (size_t)p : (size_t)a.permuted_rows[p];
+                                *reinterpret_cast<uint4*>(a.out + row * ocols + col0 + cc * 8) = val;
+                            }
+                            ++chunk;
+                        }
+                    }
                 }
                 continue;
             }
-            constexpr int kCols = kEpiCols<NT>;
+            constexpr int kCols = C::kLdCols;
             for (int j0 = jbeg; j0 < jend; j0 += kCols) {
-                uint32_t g[kCols], v[kCols];
-                tmem_ld_cols(tacc + j0, g);
-                tmem_ld_cols(tacc + NT + j0, v);
+                uint32_t gv[kCols], vv[kCols];
+                tmem_ld_cols(tacc + j0, gv);
+                tmem_ld_cols(tacc + NT + j0, vv);
                 tmem_ld_wait();
 #pragma unroll
                 for (int jj = 0; jj < kCols; ++jj) {
                     const int j = j0 + jj;
                     if (j >= jend) break;
                     const int p = t.row_start + j;
-                    const float gv = __uint_as_float(g[jj]);
+                    const float gvf = __uint_as_float(gv[jj]);
                     if (MODE == 0) {
                         float* prow = a.partials + ((size_t)split * a.R + p) * pcols;
-                        prow[f] = gv;
-                        prow[a.I + f] = __uint_as_float(v[jj]);
+                        prow[f] = gvf;
+                        prow[a.I + f] = __uint_as_float(vv[jj]);
                     } else {
                         const int r = a.permuted_rows[p];
                         float* prow = a.partials + ((size_t)split * a.R + r) * pcols;
-                        prow[f] = gv;
-                        if (f1_ok) prow[f + kBM] = __uint_as_float(v[jj]);
+                        prow[f] = gvf;
+                        if (f1_ok) prow[f + kBM] = __uint_as_float(vv[jj]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&aux->tempty[b]);
+            if (lane == 0) {
+                mbar_arrive(&aux->tempty[b]);
+                mbar_arrive(&aux->tempty2[b]);
+            }
         }
     }
 
-teardown:
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -470,12 +617,12 @@ template <int MODE, int NT>
 cudaError_t launch_mode(const CUtensorMap& tw, const CUtensorMap& ta, const FfnArgs& a, int grid,
                         cudaStream_t st)
 {
-    using C = Cfg<MODE, NT>;
+    using C = GCfg<MODE, NT>;
     auto kern = grouped_gemm_kernel<MODE, NT>;
     cudaError_t err =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (err != cudaSuccess) return err;
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, st, tw, ta, a);
+    return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, st, tw, ta, a);
 }
 
 template <int MODE>
