@@ -56,9 +56,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     ("decode", "fused_ffn"): 509_740_032 + 4_323_328,
     ("decode+e4m3", "fused_ffn"): 257_047_040 + 3_710_976,
-    # a 16-expert capture with the prefill layer's per-expert shape, x 8
-    ("prefill", "w13"): 3_510_591_488,
-    ("prefill", "w2"): 2_175_619_072,
 }
 
 # Records added to the default line (workload name, expert weight format).
@@ -465,7 +462,7 @@ def routing_bench(args, w, ctx, K, W, cpu_seconds):
     peaks, peak_kind = load_peaks()
     route_bytes = T * E * 4 + R * 8
     perm_bytes = R * 4 + (E + 1) * 4 + R * 4
-    launches = 1 + (1 if R <= 4096 else 2)  # route; one permute kernel, or count + scatter
+    launches = 1 + (1 if R <= 4096 else 3)  # route; one permute kernel, or count + scan + scatter
     ck = clocks.report()
     # The routing kernel reads the logits, the dominant traffic of the step; the
     # permutation kernels move about 1 MB and are latency-bound.

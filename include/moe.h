@@ -172,7 +172,7 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
  * threads, same device) race and may return wrong results; order them on one
  * stream. */
 #define MOE_PERMUTE_NOALLOC_MAX_ROWS (1 << 20)
-#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (2097152 + 32768 + 256)
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (2097152 + 4096 + 32768 + 256)
 moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
                                  int32_t* expert_offsets, int32_t* permuted_rows,
                                  moe_stream_t stream);

@@ -34,7 +34,7 @@ struct PermuteAux {
     int nt;                // token rows per tile (the GEMM's N tile)
     int32_t* counters;     // split-K arrival counters to zero, [n_counters]
     int n_counters;
-    int32_t* chunk_counts; // [n_chunks, E] scratch of the multi-CTA path
+    int32_t* chunk_counts; // [n_chunks + 1, E] scratch of the multi-CTA path
     // L2 prefetch of w13 for the one-launch FFN (single-CTA path, with routing):
     // the launch gets pf_units CTAs, and CTA b >= 1 prefetches the first pf_kt K
     // tiles of the gate and up blocks of w13 unit b (fused CTA b's first unit)
@@ -87,8 +87,9 @@ cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k,
                                        const PermuteAux& aux, cudaStream_t st,
                                        const CUtensorMap* pf_w13 = nullptr);
 
-// Multi-CTA path: per-chunk counts, then a per-chunk stable scatter whose CTAs
-// each scan the count table themselves (CTA 0 also writes offsets and tiles).
+// Multi-CTA path: per-chunk counts, per-expert prefixes over the chunks (and the
+// expert totals), then a per-chunk stable scatter (CTA 0 also writes offsets and
+// tiles).
 constexpr int kChunkRows = 2048;
 cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                                  int32_t* rows, const PermuteAux& aux, cudaStream_t st);

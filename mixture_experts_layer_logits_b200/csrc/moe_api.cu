@@ -104,8 +104,9 @@ Layout layout_for(const moe_shape_t& s)
     L.tiles = take((size_t)L.plan.max_tiles * sizeof(Tile));
     L.num_tiles = take(sizeof(int32_t));
     L.splits = take(2 * sizeof(int32_t));
+    // per-chunk expert counts (then prefixes), plus one row of expert totals
     const size_t n_chunks = (R + kChunkRows - 1) / kChunkRows;
-    L.chunks = take(n_chunks * (size_t)s.E * sizeof(int32_t));
+    L.chunks = take((n_chunks + 1) * (size_t)s.E * sizeof(int32_t));
     if (L.ffn) {
         size_t p13 = L.plan.s13_max > 1 ? (size_t)L.plan.s13_max * R * 2 * I : 0;
         size_t p2 = L.plan.s2_max > 1 ? (size_t)L.plan.s2_max * R * H : 0;
@@ -441,9 +442,11 @@ int moe_forward_kernel_count(moe_shape_t s)
     if (!ffn_shape_ok(s)) return 0;
     const long R = (long)s.T * s.top_k;
     const Layout L = layout_for(s);
-    if (L.fused && fused_enabled()) return (R <= kSmallRows ? 1 : 3) + 1;
-    // route(+permute) kernels, w13, [SwiGLU finalize], w2, combine
-    return (R <= kSmallRows ? 1 : 3) + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
+    // routing and permutation: one kernel, or route + count + scan + scatter
+    const int route_permute = R <= kSmallRows ? 1 : 4;
+    if (L.fused && fused_enabled()) return route_permute + 1;
+    // w13, [SwiGLU finalize], w2, combine
+    return route_permute + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
 }
 
 int moe_forward_fused(moe_shape_t s)

@@ -19,10 +19,11 @@
 namespace moe {
 namespace {
 
-// chunk count table for MOE_PERMUTE_NOALLOC_MAX_ROWS / kChunkRows chunks x 1024 experts,
-// then up to 1024 tiles (one per expert), then the tile count
+// chunk count table for MOE_PERMUTE_NOALLOC_MAX_ROWS / kChunkRows chunks x 1024 experts
+// plus its row of expert totals, then up to 1024 tiles (one per expert), then the
+// tile count
 constexpr size_t kMaxChunks = (MOE_PERMUTE_NOALLOC_MAX_ROWS + kChunkRows - 1) / kChunkRows;
-constexpr size_t kCountBytes = kMaxChunks * 1024 * sizeof(int32_t);
+constexpr size_t kCountBytes = (kMaxChunks + 1) * 1024 * sizeof(int32_t);
 constexpr size_t kTileBytes = 1024 * sizeof(Tile);
 constexpr size_t kScratchBytes = kCountBytes + kTileBytes + 256;
 static_assert(kScratchBytes == MOE_PERMUTE_NOALLOC_SCRATCH_BYTES, "header and file disagree");

@@ -118,6 +118,127 @@ __device__ __forceinline__ void warp_load_row(const float* __restrict__ row, int
     }
 }
 
+// Float -> unsigned key with the same order (-0.0 and +0.0 map to one key), and
+// back.  Key 0 stands below every non-NaN value.
+__device__ __forceinline__ uint32_t ordered_key(float f)
+{
+    const uint32_t b = __float_as_uint(f + 0.0f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t key)
+{
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// The k-th largest (k >= 1, duplicates counted) of the warp's 32 values: at most
+// k rounds of a warp max reduction, each removing the lanes that hold the max.
+__device__ __forceinline__ float warp_kth_largest(float x, int k)
+{
+    uint32_t key = ordered_key(x);
+    int left = k;
+    for (;;) {
+        const uint32_t m = __reduce_max_sync(kFull, key);
+        left -= __popc(__ballot_sync(kFull, key == m));
+        if (left <= 0) return key_value(m);
+        if (key == m) key = 0;
+    }
+}
+
+// Sorts the candidates cand[0 .. total) (total <= 32, distinct experts) by (logit
+// desc, expert asc) and leaves the j-th in lane j: (my_l, my_id).
+__device__ __forceinline__ void sort_candidates(int total, int lane, const float2* cand,
+                                                float& my_l, int& my_id)
+{
+    float cv = -INFINITY;
+    int ci = kNoIndex - lane;  // distinct sentinels rank after every expert
+    if (lane < total) {
+        const float2 cc = cand[lane];
+        cv = cc.x;
+        ci = __float_as_int(cc.y);
+    }
+    __syncwarp();  // cand may be rewritten by this warp's next token
+    // usually about k candidates: then lanes 0..15 hold all of them and a
+    // half-warp network (10 stages instead of 15) orders them the same way
+    if (total <= 16)
+        warp_sort_keys<16>(cv, ci, lane);
+    else
+        warp_sort_keys<32>(cv, ci, lane);
+    my_l = cv;
+    my_id = ci;
+}
+
+// Softmax over the selected logits (lane j holds the j-th; l_0 is the largest)
+// and the outputs.  The sum is a fixed xor-tree over lanes 0..15 (lanes >= k
+// contribute 0), so it is deterministic.
+__device__ __forceinline__ void write_selection(float my_l, int my_id, int k, int lane,
+                                                int32_t* __restrict__ ids,
+                                                float* __restrict__ weights, int* ids_s)
+{
+    const float l0 = __shfl_sync(kFull, my_l, 0);
+    const float ex = (lane < k) ? expf(my_l - l0) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    sum = __shfl_sync(kFull, sum, 0);
+    if (lane < k) {
+        if (ids) {
+            ids[lane] = my_id;
+            weights[lane] = ex / sum;
+        }
+        if (ids_s) ids_s[lane] = my_id;
+    }
+}
+
+// Exact selection when more than 32 experts reach the threshold (ties, -inf
+// rows): the k winners one by one with a warp arg-max.
+template <int V, bool VEC>
+__device__ __forceinline__ void select_exhaustive(const float (&v)[V], int E, int k, int lane,
+                                                  float& my_l, int& my_id)
+{
+    uint32_t taken = 0;
+    // best not-yet-taken value of this lane; slots ascend with the expert, so a
+    // strict '>' keeps the lower expert on equal values
+    auto lane_best = [&](float& bv, int& bi) {
+        bv = -INFINITY;
+        bi = kNoIndex;
+#pragma unroll
+        for (int m = 0; m < V; ++m) {
+            const int e = slot_expert<V, VEC>(m, lane);
+            const bool ok = e < E && !((taken >> m) & 1u);
+            if (ok && (bi == kNoIndex || v[m] > bv)) {
+                bv = v[m];
+                bi = e;
+            }
+        }
+    };
+    float bv;
+    int bi;
+    lane_best(bv, bi);
+    for (int j = 0; j < k; ++j) {
+        float wv = bv;
+        int wi = bi;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(kFull, wv, off);
+            const int oi = __shfl_xor_sync(kFull, wi, off);
+            if (key_before(ov, oi, wv, wi)) {
+                wv = ov;
+                wi = oi;
+            }
+        }
+        if (lane == j) {
+            my_l = wv;
+            my_id = wi;
+        }
+        const int owner = VEC ? (wi & 127) >> 2 : (wi & 31);
+        if (owner == lane) {  // the owner drops the winner and finds its next best
+            const int slot = VEC ? (wi >> 7) * 4 + (wi & 3) : (wi >> 5);
+            taken |= 1u << slot;
+            lane_best(bv, bi);
+        }
+    }
+}
+
 template <int V, bool VEC>
 __device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, int k, int lane,
                                                   int32_t* __restrict__ ids,
@@ -165,81 +286,54 @@ __device__ __forceinline__ void warp_select_token(const float (&v)[V], int E, in
             }
         }
         __syncwarp();
-        float cv = -INFINITY;
-        int ci = kNoIndex - lane;  // distinct sentinels rank after every expert
-        if (lane < total) {
-            const float2 cc = cand[lane];
-            cv = cc.x;
-            ci = __float_as_int(cc.y);
-        }
-        __syncwarp();  // cand may be rewritten by this warp's next token
-        // usually about k candidates: then lanes 0..15 hold all of them and a
-        // half-warp network (10 stages instead of 15) orders them the same way
-        if (total <= 16)
-            warp_sort_keys<16>(cv, ci, lane);
-        else
-            warp_sort_keys<32>(cv, ci, lane);
-        my_l = cv;
-        my_id = ci;
+        sort_candidates(total, lane, cand, my_l, my_id);
     } else {
-        uint32_t taken = 0;
-        // best not-yet-taken value of this lane; slots ascend with the expert, so a
-        // strict '>' keeps the lower expert on equal values
-        auto lane_best = [&](float& bv, int& bi) {
-            bv = -INFINITY;
-            bi = kNoIndex;
-#pragma unroll
-            for (int m = 0; m < V; ++m) {
-                const int e = slot_expert<V, VEC>(m, lane);
-                const bool ok = e < E && !((taken >> m) & 1u);
-                if (ok && (bi == kNoIndex || v[m] > bv)) {
-                    bv = v[m];
-                    bi = e;
-                }
-            }
-        };
-        float bv;
-        int bi;
-        lane_best(bv, bi);
-        for (int j = 0; j < k; ++j) {
-            float wv = bv;
-            int wi = bi;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(kFull, wv, off);
-                const int oi = __shfl_xor_sync(kFull, wi, off);
-                if (key_before(ov, oi, wv, wi)) {
-                    wv = ov;
-                    wi = oi;
-                }
-            }
-            if (lane == j) {
-                my_l = wv;
-                my_id = wi;
-            }
-            const int owner = VEC ? (wi & 127) >> 2 : (wi & 31);
-            if (owner == lane) {  // the owner drops the winner and finds its next best
-                const int slot = VEC ? (wi >> 7) * 4 + (wi & 3) : (wi >> 5);
-                taken |= 1u << slot;
-                lane_best(bv, bi);
-            }
-        }
+        select_exhaustive<V, VEC>(v, E, k, lane, my_l, my_id);
     }
-    // softmax over the selected logits; l_0 is the largest.  The sum is a fixed
-    // xor-tree over lanes 0..15 (lanes >= k contribute 0), so it is deterministic.
-    const float l0 = __shfl_sync(kFull, my_l, 0);
-    const float ex = (lane < k) ? expf(my_l - l0) : 0.f;
-    float sum = ex;
+    write_selection(my_l, my_id, k, lane, ids, weights, ids_s);
+}
+
+// warp_select_token for a row that is also staged in shared memory (rowf[e] =
+// logit of expert e; float4 slot layout, E % 4 == 0).  The threshold comes from
+// warp max reductions, each lane marks its slots that reach it in a bit mask,
+// and only the marked slots are read back (from shared memory) as candidates.
+template <int V, bool FULL>
+__device__ __forceinline__ void warp_select_staged(const float (&v)[V], const float* rowf, int E,
+                                                   int k, int lane, int32_t* __restrict__ ids,
+                                                   float* __restrict__ weights, float2* cand)
+{
+    float mv = -INFINITY;
 #pragma unroll
-    for (int off = 1; off < 16; off <<= 1) sum += __shfl_xor_sync(kFull, sum, off);
-    sum = __shfl_sync(kFull, sum, 0);
-    if (lane < k) {
-        if (ids) {
-            ids[lane] = my_id;
-            weights[lane] = ex / sum;
-        }
-        if (ids_s) ids_s[lane] = my_id;
+    for (int m = 0; m < V; ++m) mv = fmaxf(mv, v[m]);
+    const float tau = warp_kth_largest(mv, k);
+    uint32_t mask = 0;
+#pragma unroll
+    for (int m = 0; m < V; ++m)
+        if ((FULL || slot_expert<V, true>(m, lane) < E) && v[m] >= tau) mask |= 1u << m;
+    const int c = __popc(mask);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += n;
     }
+    const int total = __shfl_sync(kFull, incl, 31);
+    float my_l = 0.f;
+    int my_id = 0;
+    if (total <= 32) {
+        int pos = incl - c;
+        while (mask) {
+            const int m = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int e = slot_expert<V, true>(m, lane);
+            cand[pos++] = make_float2(rowf[e], __int_as_float(e));
+        }
+        __syncwarp();
+        sort_candidates(total, lane, cand, my_l, my_id);
+    } else {
+        select_exhaustive<V, true>(v, E, k, lane, my_l, my_id);
+    }
+    write_selection(my_l, my_id, k, lane, ids, weights, nullptr);
 }
 
 template <int V, bool VEC>
@@ -373,6 +467,73 @@ __global__ void __launch_bounds__(256, 4) route_kernel(const float* __restrict__
                              weights + (size_t)t * k, nullptr, cand[threadIdx.x >> 5]);
 }
 
+// Routing with many experts per token (E = 32 V logits, V >= 16, E % 4 == 0):
+// persistent warps, warp w of the grid routing tokens w, w + W, ... (W = all warps).
+// A token row is E * 4 bytes; each lane copies its own 16-byte pieces of it (the
+// float4 slot layout of warp_load_row: piece m of lane l = experts 128 m + 4 l ..)
+// with cp.async into the warp's ring of kRouteDepth rows in shared memory,
+// kRouteDepth - 1 tokens ahead of the one being selected (one ahead: a second
+// row per warp measured slower than the third CTA per SM it costs), and reads
+// back only
+// what it copied itself -- its own cp.async.wait_group makes those visible, so no
+// barrier is involved.  The logits of later tokens stream from HBM while the
+// current one is selected.
+constexpr int kRouteWarps = 8;
+constexpr int kRouteDepth = 2;
+
+template <int V, bool FULL>
+__global__ void __launch_bounds__(kRouteWarps * 32, 3)
+    route_stream_kernel(const float* __restrict__ logits, int T, int E, int k,
+                        int32_t* __restrict__ ids, float* __restrict__ weights)
+{
+    static_assert(V % 4 == 0, "float4 slots");
+    constexpr int kPieces = V / 4;  // 16-byte pieces per lane and row
+    extern __shared__ float4 ring[];  // [kRouteWarps][kRouteDepth][kPieces][32]
+    __shared__ float2 cand[kRouteWarps][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float4* my = ring + (size_t)warp * kRouteDepth * kPieces * 32;
+    pdl_wait();
+    pdl_launch_dependents();
+    const uint64_t pol = l2_policy_evict_first();  // each logit is read once
+    const int W = gridDim.x * kRouteWarps;
+    const int w0 = blockIdx.x * kRouteWarps + warp;
+    auto issue = [&](int t, int slot) {
+        if (t < T) {
+            const float* row = logits + (size_t)t * E;
+#pragma unroll
+            for (int m = 0; m < kPieces; ++m) {
+                const int e = m * 128 + lane * 4;
+                if (e < E)
+                    cp_async_16_hint(smem_u32(my + (slot * kPieces + m) * 32 + lane), row + e, pol);
+            }
+        }
+        cp_async_commit();  // one group per token, empty or not
+    };
+#pragma unroll
+    for (int d = 0; d < kRouteDepth - 1; ++d) issue(w0 + d * W, d);
+    int slot = 0;
+    for (int t = w0; t < T; t += W) {
+        // the slot refilled now held the previous token, whose values were
+        // consumed by its selection
+        issue(t + (kRouteDepth - 1) * W, (slot + kRouteDepth - 1) % kRouteDepth);
+        cp_async_wait<kRouteDepth - 1>();  // this token's pieces have landed
+        float v[V];
+#pragma unroll
+        for (int m = 0; m < kPieces; ++m) {
+            float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            if (m * 128 + lane * 4 < E) q = my[(slot * kPieces + m) * 32 + lane];
+            v[4 * m] = q.x;
+            v[4 * m + 1] = q.y;
+            v[4 * m + 2] = q.z;
+            v[4 * m + 3] = q.w;
+        }
+        warp_select_staged<V, FULL>(v, reinterpret_cast<const float*>(my + slot * kPieces * 32), E, k,
+                              lane, ids + (size_t)t * k, weights + (size_t)t * k, cand[warp]);
+        slot = (slot + 1) % kRouteDepth;
+    }
+    cp_async_wait<0>();
+}
+
 // One CTA: (route) + count + scan + stable scatter + tile list, for T*k <= kSmallRows.
 // CTAs 1.. of the single-CTA permutation launch when the one-launch FFN follows
 // (aux.pf_units > 0).  Each routes the T tokens again (ids into shared memory
@@ -498,70 +659,96 @@ __global__ void __launch_bounds__(1024) chunk_count_kernel(const int32_t* __rest
     for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = hist[e];
 }
 
-// One CTA per chunk of kChunkRows expanded rows.  Every CTA reads the whole
-// per-chunk count table (kept in L2) to get, for each expert e, the rows of e in
-// all chunks (-> the exclusive scan over experts, expert_offsets) and in the
-// chunks before its own (-> where its own rows of e start); then it ranks its
-// rows stably with per-warp tables and scatters them.  CTA 0 also writes
-// expert_offsets and the tile list.
+// After chunk_count_kernel, for experts 32 b .. 32 b + 31 (CTA b, lane = expert):
+// warp w walks the chunks [w L, (w + 1) L) (L = ceil(n_chunks / 32)) of its
+// expert, the 32 warps' sums are scanned in shared memory, and counts[c][e] is
+// overwritten with P[c][e] = the rows of e in the chunks before c.  Row n_chunks
+// of the table receives the expert's total.  Every chunk read is coalesced over
+// the 32 experts of a warp.
+__global__ void __launch_bounds__(1024, 1)
+    chunk_prefix_kernel(int32_t* __restrict__ counts, int n_chunks, int E)
+{
+    __shared__ int part[32][33];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.x * 32 + lane;
+    const int L = (n_chunks + 31) / 32;
+    const int c0 = min(n_chunks, warp * L), c1 = min(n_chunks, c0 + L);
+    int sum = 0;
+    if (e < E)
+        for (int c = c0; c < c1; ++c) sum += __ldcg(counts + (size_t)c * E + e);
+    part[warp][lane] = sum;
+    __syncthreads();
+    int pre = 0;
+    for (int w = 0; w < warp; ++w) pre += part[w][lane];
+    if (e < E) {
+        int run = pre;
+        for (int c = c0; c < c1; ++c) {
+            const int v = __ldcg(counts + (size_t)c * E + e);
+            counts[(size_t)c * E + e] = run;
+            run += v;
+        }
+        if (warp == 31) counts[(size_t)n_chunks * E + e] = run;  // the expert's total
+    }
+}
+
+constexpr int kRankWarps = 8;
+
+// One CTA per chunk of kChunkRows expanded rows, after chunk_prefix_kernel.  The
+// expert totals (row n_chunks of the table) give expert_offsets by an exclusive
+// scan over experts (CTA 0 also writes them and the tile list); base[e] =
+// expert_offsets[e] + P[chunk][e] is where the chunk's first row of expert e
+// goes.  The chunk's rows are ranked stably with per-warp count tables (a warp's
+// rows in order, warps in order) and scattered.
 __global__ void __launch_bounds__(1024, 1)
     chunk_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, int n_chunks,
-                         const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         const int32_t* __restrict__ prefix, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ rows_out, PermuteAux aux)
 {
     extern __shared__ int smem[];
     __shared__ int sums[32];
     int* ids_s = smem;                 // kChunkRows
-    int* table = smem + kChunkRows;    // [32][E]
+    int* table = smem + kChunkRows;    // [kRankWarps][E]
     const int warp = threadIdx.x >> 5;
     pdl_wait();
     pdl_launch_dependents();
     const int c0 = blockIdx.x * kChunkRows, n = min(kChunkRows, R - c0);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) ids_s[i] = ids[c0 + i];
-    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) table[i] = 0;
-
-    // per expert: rows in all chunks and rows in the chunks before this one; the
-    // loads of a batch are all issued before they are used
     const bool owns = threadIdx.x < E;
     const int e = threadIdx.x;
-    int total_e = 0, before_e = 0;
-    if (owns) {
-        constexpr int kBatch = 16;
-        for (int cb = 0; cb < n_chunks; cb += kBatch) {
-            int vals[kBatch];
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i)
-                vals[i] = (cb + i < n_chunks) ? __ldcg(counts + (size_t)(cb + i) * E + e) : 0;
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-                total_e += vals[i];
-                if (cb + i < (int)blockIdx.x) before_e += vals[i];
-            }
-        }
-    }
+    // the three loads are independent: issue them before anything waits
+    const int total_e = owns ? __ldcg(prefix + (size_t)n_chunks * E + e) : 0;
+    const int pre_e = owns ? __ldcg(prefix + (size_t)blockIdx.x * E + e) : 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) ids_s[i] = ids[c0 + i];
+    for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) table[i] = 0;
     int total;
-    const int off = block_exclusive_scan(owns ? total_e : 0, sums, total);
+    const int off = block_exclusive_scan(total_e, sums, total);  // ends with a barrier
     if (blockIdx.x == 0) {
         if (owns) offsets[e] = off;
         if (threadIdx.x == 0) offsets[E] = total;
         write_tiles_and_reset(owns, e, total_e, off, aux, sums);
     }
-    __syncthreads();  // ids_s and the zeroed table are complete
 
-    constexpr int per_warp = kChunkRows / 32;
+    // kRankWarps warps rank the chunk's rows, kChunkRows / kRankWarps each, in
+    // order: fewer count rows to clear and to scan than one per warp of the CTA
+    constexpr int per_warp = kChunkRows / kRankWarps;
     const int r0 = min(n, warp * per_warp), r1 = min(n, r0 + per_warp);
-    warp_count(ids_s, r0, r1, table + warp * E);
+    if (warp < kRankWarps) warp_count(ids_s, r0, r1, table + warp * E);
     __syncthreads();
     if (owns) {
-        int run = off + before_e;
-        for (int w = 0; w < 32; ++w) {
-            const int v = table[w * E + e];
+        // the ranking warps' counts of expert e, read before any is overwritten
+        int v[kRankWarps];
+#pragma unroll
+        for (int w = 0; w < kRankWarps; ++w) v[w] = table[w * E + e];
+        int run = off + pre_e;
+#pragma unroll
+        for (int w = 0; w < kRankWarps; ++w) {
             table[w * E + e] = run;
-            run += v;
+            run += v[w];
         }
     }
     __syncthreads();
-    warp_scatter(ids_s, r0, r1, c0, table + warp * E, rows_out);
+    if (warp < kRankWarps) warp_scatter(ids_s, r0, r1, c0, table + warp * E, rows_out);
 }
 
 __global__ void __launch_bounds__(1024) build_tiles_kernel(const int32_t* __restrict__ offsets,
@@ -595,6 +782,26 @@ template <int V>
 static cudaError_t launch_route_v(bool vec, const float* logits, int T, int E, int k, int32_t* ids,
                                   float* weights, cudaStream_t st)
 {
+    if constexpr (V >= 16) {
+        if (vec) {
+            const size_t smem = sizeof(float) * (size_t)kRouteWarps * kRouteDepth * 32 * V;
+            int dev = 0, sms = 148;
+            if (cudaGetDevice(&dev) == cudaSuccess)
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            // three CTAs per SM (64 KB of rings each at V = 32), no more than the tokens need
+            const int want = (T + kRouteWarps - 1) / kRouteWarps;
+            const int grid = want < 3 * sms ? want : 3 * sms;
+            auto go = [&](auto kern) {
+                cudaError_t err = cudaFuncSetAttribute(
+                    kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (err != cudaSuccess) return err;
+                return launch(kern, dim3(grid), dim3(kRouteWarps * 32), smem, st, logits, T, E, k,
+                              ids, weights);
+            };
+            return E == 32 * V ? go(route_stream_kernel<V, true>)
+                               : go(route_stream_kernel<V, false>);
+        }
+    }
     const dim3 grid((T + 7) / 8), block(256);
     if (vec && V >= 4)
         return launch(route_kernel<V, (V >= 4)>, grid, block, 0, st, logits, T, E, k, ids, weights);
@@ -657,7 +864,7 @@ cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k,
 #undef MOE_SMALL
 }
 
-size_t large_permute_smem(int E) { return sizeof(int) * (size_t)(kChunkRows + 32 * E); }
+size_t large_permute_smem(int E) { return sizeof(int) * (size_t)(kChunkRows + kRankWarps * E); }
 
 cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                                  int32_t* rows, const PermuteAux& aux, cudaStream_t st)
@@ -666,6 +873,9 @@ cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_
     const int n_chunks = (R + kChunkRows - 1) / kChunkRows;
     cudaError_t err = launch(chunk_count_kernel, dim3(n_chunks), dim3(1024), sizeof(int) * E, st,
                              ids, R, E, aux.chunk_counts);
+    if (err != cudaSuccess) return err;
+    err = launch(chunk_prefix_kernel, dim3((E + 31) / 32), dim3(1024), 0, st, aux.chunk_counts,
+                 n_chunks, E);
     if (err != cudaSuccess) return err;
     const size_t smem = large_permute_smem(E);
     err = cudaFuncSetAttribute(chunk_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
