@@ -67,7 +67,8 @@ typedef enum {
     MOE_ERR_MISALIGNED = 3,
     MOE_ERR_WORKSPACE_TOO_SMALL = 4,
     MOE_ERR_CUDA = 5,
-    MOE_ERR_DEVICE_TIMEOUT = 6
+    MOE_ERR_DEVICE_TIMEOUT = 6,
+    MOE_ERR_DEVICE_BOUNDS = 7   /* debug build only: see moe_device_status */
 } moe_status_t;
 
 /* T tokens, E experts, top_k, H hidden, I intermediate (H, I unused by route/permute). */
@@ -230,7 +231,14 @@ int moe_forward_fused(moe_shape_t shape);
 
 /* Waits for `stream`, then reads and clears the device error word kept in the
  * workspace.  MOE_ERR_DEVICE_TIMEOUT means a kernel gave up on a bounded
- * intra-kernel wait (its outputs for that call are then unspecified). */
+ * intra-kernel wait (its outputs for that call are then unspecified).
+ * MOE_ERR_DEVICE_BOUNDS comes only from the debug build of the library
+ * (libmoe_debug.so, compiled with MOE_DEBUG): one of its kernels read an index
+ * out of range from its inputs -- an expert id outside [0, E) given to
+ * moe_permute, expert offsets outside [0, T*k] or a permuted row outside
+ * [0, T*k) given to moe_grouped_ffn -- and skipped (or redirected to index 0)
+ * the access it would have made; that call's outputs are unspecified.  The
+ * release build does not check these out-of-contract inputs. */
 moe_status_t moe_device_status(void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* Static description of a status code. */

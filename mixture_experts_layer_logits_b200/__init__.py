@@ -22,13 +22,20 @@ __all__ = [
     "moe_device_status", "library_path", "load_library",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED_SHAPE", "MOE_ERR_MISALIGNED",
     "MOE_ERR_WORKSPACE_TOO_SMALL", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
+    "MOE_ERR_DEVICE_BOUNDS", "debug_library_path",
 ]
 
 (MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_MISALIGNED,
- MOE_ERR_WORKSPACE_TOO_SMALL, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT) = range(7)
+ MOE_ERR_WORKSPACE_TOO_SMALL, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT,
+ MOE_ERR_DEVICE_BOUNDS) = range(8)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libmoe.so")
+# libmoe_debug.so: the same library with the kernels' input-index checks compiled
+# in (moe_device_status then reports MOE_ERR_DEVICE_BOUNDS); MOE_LIBRARY=debug in
+# the environment selects it at import.
+debug_library_path = os.path.join(_HERE, "libmoe_debug.so")
+library_path = (debug_library_path if os.environ.get("MOE_LIBRARY", "") == "debug"
+                else os.path.join(_HERE, "libmoe.so"))
 
 
 class Shape(ctypes.Structure):
@@ -56,7 +63,7 @@ _vp = ctypes.c_void_p
 
 
 def load_library():
-    """Load libmoe.so (raises OSError if it was not built)."""
+    """Load the library at library_path (raises OSError if it was not built)."""
     global _lib
     if _lib is not None:
         return _lib

@@ -435,8 +435,9 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < C::kGIters; ++i) {
                     const int j = (g + i * kGGatherThreads) >> 3;
-                    off[i] = j < t.rows ? (a.permuted_rows[t.row_start + j] / a.k) * a.H + (g & 7) * 8
-                                        : -1;
+                    int r = j < t.rows ? a.permuted_rows[t.row_start + j] : -1;
+                    if (r >= 0 && !debug_in_range(r, 0, a.R, a.err)) r = 0;  // debug build
+                    off[i] = r >= 0 ? (r / a.k) * a.H + (g & 7) * 8 : -1;
                 }
                 cur_tile = tile;
             }
@@ -560,8 +561,10 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
                                 const int p = t.row_start + jbeg + c + jj;
                                 const uint4 val = *reinterpret_cast<const uint4*>(
                                     buf + jj * C::kRowBytes + cc * 16);
-                                const size_t row = MODE == 0 ? (size_t)p : (size_t)a.permuted_rows[p];
-                                *reinterpret_cast<uint4*>(a.out + row * ocols + col0 + cc * 8) = val;
+                                const int row = MODE == 0 ? p : a.permuted_rows[p];
+                                if (debug_in_range(row, 0, a.R, a.err))
+                                    *reinterpret_cast<uint4*>(a.out + (size_t)row * ocols + col0 +
+                                                              cc * 8) = val;
                             }
                             ++chunk;
                         }
@@ -587,6 +590,7 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
                         prow[a.I + f] = __uint_as_float(vv[jj]);
                     } else {
                         const int r = a.permuted_rows[p];
+                        if (!debug_in_range(r, 0, a.R, a.err)) continue;
                         float* prow = a.partials + ((size_t)split * a.R + r) * pcols;
                         prow[f] = gvf;
                         if (f1_ok) prow[f + kBM] = __uint_as_float(vv[jj]);

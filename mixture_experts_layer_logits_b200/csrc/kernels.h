@@ -15,6 +15,30 @@ namespace moe {
 // value counts as an error.
 constexpr int32_t kDeviceErrorMagic = 0x4D4F4554;
 
+// Value a kernel of the debug build (compiled with MOE_DEBUG) stores in the error
+// word when an index read from its inputs -- an expert id, an expert offset, a
+// permuted row -- is out of range; the access it would have made is skipped or
+// redirected to index 0.
+constexpr int32_t kDeviceBoundsMagic = 0x4D4F4542;
+
+#ifdef MOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+// Debug build: true when lo <= v < hi; otherwise records kDeviceBoundsMagic in
+// *err (when err is not null) and returns false.  Release build: always true,
+// and the check compiles away.
+__device__ __forceinline__ bool debug_in_range(long long v, long long lo, long long hi,
+                                               int32_t* err)
+{
+    if constexpr (!kDebugChecks) return true;
+    const bool ok = v >= lo && v < hi;
+    if (!ok && err) atomicExch(err, kDeviceBoundsMagic);
+    return ok;
+}
+
 // One tile of the grouped GEMMs: `rows` (1..NT) consecutive permuted rows of one
 // expert, starting at permuted position `row_start`.  `first` is the index of the
 // expert's first tile and `count` its number of tiles.
@@ -35,6 +59,8 @@ struct PermuteAux {
     int32_t* counters;     // split-K arrival counters to zero, [n_counters]
     int n_counters;
     int32_t* chunk_counts; // [n_chunks + 1, E] scratch of the multi-CTA path
+    int32_t* err;          // the error word (debug-build index checks); may be null
+    int max_tiles;         // entries of `tiles`
     // L2 prefetch of w13 for the one-launch FFN (single-CTA path, with routing):
     // the launch gets pf_units CTAs, and CTA b >= 1 prefetches the first pf_kt K
     // tiles of the gate and up blocks of w13 unit b (fused CTA b's first unit)
@@ -96,7 +122,7 @@ cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_
 size_t large_permute_smem(int E);
 
 // Tile list from expert_offsets alone (moe_grouped_ffn called on its own).
-cudaError_t launch_build_tiles(const int32_t* offsets, int E, const PermuteAux& aux,
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, int R, const PermuteAux& aux,
                                cudaStream_t st);
 
 struct FfnPlan {

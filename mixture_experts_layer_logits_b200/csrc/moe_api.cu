@@ -162,6 +162,8 @@ PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
     a.counters = L.fused ? at<int32_t>(ws, L.counters) : nullptr;
     a.n_counters = L.fused ? L.n_counters : 0;
     a.chunk_counts = at<int32_t>(ws, L.chunks);
+    a.err = at<int32_t>(ws, L.err);
+    a.max_tiles = L.plan.max_tiles;
     a.pf_units = 0;
     a.pf_fb13 = a.pf_I = a.pf_kt = 0;
     (void)s;
@@ -290,7 +292,8 @@ moe_status_t moe_grouped_ffn(const moe_bf16_t* x, const moe_bf16_t* w13, const m
     if (ws_bytes < moe_workspace_size(s)) return MOE_ERR_WORKSPACE_TOO_SMALL;
     const Layout L = layout_for(s);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    moe_status_t r = cuda_status(launch_build_tiles(expert_offsets, s.E, make_aux(ws, L, s), st));
+    moe_status_t r = cuda_status(
+        launch_build_tiles(expert_offsets, s.E, s.T * s.top_k, make_aux(ws, L, s), st));
     if (r != MOE_OK) return r;
     return run_ffn(x, w13, w2, permuted_rows, s, y, ws, L, st);
 }
@@ -469,7 +472,9 @@ moe_status_t moe_device_status(void* ws, size_t ws_bytes, moe_stream_t stream)
     e = cudaMemcpyAsync(ws, &zero, sizeof zero, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_status(e);
-    return v == kDeviceErrorMagic ? MOE_ERR_DEVICE_TIMEOUT : MOE_OK;
+    return v == kDeviceErrorMagic    ? MOE_ERR_DEVICE_TIMEOUT
+           : v == kDeviceBoundsMagic ? MOE_ERR_DEVICE_BOUNDS
+                                     : MOE_OK;
 }
 
 moe_status_t moe_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned limit_us,
@@ -491,6 +496,8 @@ const char* moe_status_string(moe_status_t status)
     case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case MOE_ERR_CUDA: return "CUDA error (see moe_last_cuda_error)";
     case MOE_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case MOE_ERR_DEVICE_BOUNDS:
+        return "a debug-build kernel found an input index out of range (the access was skipped)";
     }
     return "unknown status";
 }

@@ -393,6 +393,11 @@ __device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int coun
     }
     int total;
     const int start = block_exclusive_scan(n, sums, total);
+    // debug build: never past the tile array (only out-of-contract offsets can
+    // ask for more tiles than it holds)
+    if (n > 0 && !debug_in_range(start + n - 1, 0, aux.max_tiles, aux.err))
+        n = max(0, aux.max_tiles - start);
+    if (kDebugChecks) total = min(total, aux.max_tiles);
     for (int i = 0; i < n; ++i) {
         Tile t;
         t.expert = e;
@@ -611,7 +616,10 @@ __global__ void __launch_bounds__(1024, 1)
             for (int m = 0; m < V; ++m) v[m] = nv[m];
         }
     } else {
-        for (int r = threadIdx.x; r < R; r += blockDim.x) ids_s[r] = ids[r];
+        for (int r = threadIdx.x; r < R; r += blockDim.x) {
+            const int e = ids[r];
+            ids_s[r] = debug_in_range(e, 0, E, aux.err) ? e : 0;
+        }
     }
     // counting warps: as many as there are 32-row groups, up to 32
     const int W = min(32, (R + 31) / 32);
@@ -646,7 +654,8 @@ __global__ void __launch_bounds__(1024, 1)
 }
 
 __global__ void __launch_bounds__(1024) chunk_count_kernel(const int32_t* __restrict__ ids, int R,
-                                                           int E, int32_t* __restrict__ counts)
+                                                           int E, int32_t* __restrict__ counts,
+                                                           int32_t* err)
 {
     extern __shared__ int hist[];
     pdl_wait();
@@ -654,7 +663,10 @@ __global__ void __launch_bounds__(1024) chunk_count_kernel(const int32_t* __rest
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int r0 = blockIdx.x * kChunkRows, r1 = min(R, r0 + kChunkRows);
-    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) atomicAdd(&hist[ids[r]], 1);
+    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+        const int e = ids[r];
+        atomicAdd(&hist[debug_in_range(e, 0, E, err) ? e : 0], 1);
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = hist[e];
 }
@@ -719,7 +731,10 @@ __global__ void __launch_bounds__(1024, 1)
     // the three loads are independent: issue them before anything waits
     const int total_e = owns ? __ldcg(prefix + (size_t)n_chunks * E + e) : 0;
     const int pre_e = owns ? __ldcg(prefix + (size_t)blockIdx.x * E + e) : 0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) ids_s[i] = ids[c0 + i];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int id = ids[c0 + i];
+        ids_s[i] = debug_in_range(id, 0, E, aux.err) ? id : 0;
+    }
     for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) table[i] = 0;
     int total;
     const int off = block_exclusive_scan(total_e, sums, total);  // ends with a barrier
@@ -752,15 +767,18 @@ __global__ void __launch_bounds__(1024, 1)
 }
 
 __global__ void __launch_bounds__(1024) build_tiles_kernel(const int32_t* __restrict__ offsets,
-                                                           int E, PermuteAux aux)
+                                                           int E, int R, PermuteAux aux)
 {
     __shared__ int sums[32];
     pdl_wait();
     pdl_launch_dependents();
     const bool owns = threadIdx.x < E;
     const int e = threadIdx.x;
-    const int off = owns ? offsets[e] : 0;
-    const int cnt = owns ? offsets[e + 1] - off : 0;
+    int off = owns ? offsets[e] : 0;
+    int cnt = owns ? offsets[e + 1] - off : 0;
+    // debug build: an expert's rows must lie inside [0, R); otherwise it gets no tile
+    if (owns && !(debug_in_range(off, 0, R + 1, aux.err) && debug_in_range(cnt, 0, R - off + 1, aux.err)))
+        off = cnt = 0;
     write_tiles_and_reset(owns, e, cnt, off, aux, sums);
 }
 
@@ -872,7 +890,7 @@ cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_
     const int R = T * k;
     const int n_chunks = (R + kChunkRows - 1) / kChunkRows;
     cudaError_t err = launch(chunk_count_kernel, dim3(n_chunks), dim3(1024), sizeof(int) * E, st,
-                             ids, R, E, aux.chunk_counts);
+                             ids, R, E, aux.chunk_counts, aux.err);
     if (err != cudaSuccess) return err;
     err = launch(chunk_prefix_kernel, dim3((E + 31) / 32), dim3(1024), 0, st, aux.chunk_counts,
                  n_chunks, E);
@@ -885,10 +903,10 @@ cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_
                   (const int32_t*)aux.chunk_counts, offsets, rows, aux);
 }
 
-cudaError_t launch_build_tiles(const int32_t* offsets, int E, const PermuteAux& aux,
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, int R, const PermuteAux& aux,
                                cudaStream_t st)
 {
-    return launch(build_tiles_kernel, dim3(1), dim3(1024), 0, st, offsets, E, aux);
+    return launch(build_tiles_kernel, dim3(1), dim3(1024), 0, st, offsets, E, R, aux);
 }
 
 }  // namespace moe

@@ -198,7 +198,7 @@ def test_device_status_validation(lib):
 
 def test_status_strings(lib):
     seen = set()
-    for code in range(7):
+    for code in range(8):
         s = lib.moe_status_string(code).decode()
         assert s and s not in seen
         seen.add(s)
