@@ -151,11 +151,11 @@ def stage_work(w, n_touched, weights="bf16"):
         "w2": dict(bytes=n_touched * (H * I * wb + s2) + R * I * 2 + R * H * 2,
                    flops=2 * R * H * I),
         "combine": dict(bytes=R * H * 2 + R * 4 + T * H * 2, flops=0),
-        # w13 + w2 + combine as one launch: act and y never need to reach HBM, so
-        # the algorithmic bytes are the touched weights, x, the routing weights and
-        # permuted rows, and out
+        # routing + w13 + w2 + combine as one launch: act and y never need to reach
+        # HBM, so the algorithmic bytes are the touched weights, x, the routing
+        # weights and permuted rows, out, and the routing's logits and outputs
         "fused_ffn": dict(bytes=n_touched * (3 * I * H * wb + s13 + s2) + T * H * 2 + R * 8 +
-                          T * H * 2,
+                          T * H * 2 + T * E * 4 + R * 12 + (E + 1) * 4,
                           flops=2 * R * 2 * I * H + 2 * R * H * I),
     }
 
@@ -606,8 +606,8 @@ def layer_bench(args, w, weights, ctx, K, W, cpu_seconds):
         fwd(sev[i])
     barrier()
     fused = e4m3 or moe.moe_forward_fused(T, E, k, H, I)
-    if fused:  # events 2..4 all follow the one FFN + combine launch
-        spans = {"route_permute": (0, 1), "fused_ffn": (1, 4)}
+    if fused:  # one launch: routing, FFN and combine (events 1..4 around it)
+        spans = {"fused_ffn": (0, 4)}
     else:
         spans = {"route_permute": (0, 1), "w13": (1, 2), "w2": (2, 3), "combine": (3, 4)}
     stage_ms = {n: statistics.mean(sev[i][a].elapsed_time(sev[i][b]) for i in range(KB))
@@ -673,8 +673,8 @@ def layer_bench(args, w, weights, ctx, K, W, cpu_seconds):
                "kind": "oracle", "sample": f"{sample} in {dt:.1f} s"}
     if rank != 0:
         return None
-    # E4M3 weights always take the one-launch FFN: routing + permute, then the FFN
-    launches = 2 if e4m3 else moe.moe_forward_kernel_count(T, E, k, H, I)
+    # E4M3 weights always take the one-launch path (routing included)
+    launches = 1 if e4m3 else moe.moe_forward_kernel_count(T, E, k, H, I)
     return {
         "metric": metric_name(w),
         "value": round(weak_scaling_value(world, T, ms), 2),

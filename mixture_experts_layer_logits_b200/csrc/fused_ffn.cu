@@ -64,6 +64,7 @@
 #include <cuda_fp16.h>
 
 #include "gemm_common.cuh"
+#include "route_common.cuh"
 
 namespace moe {
 
@@ -76,22 +77,26 @@ constexpr int kMaxSplits = 8;   // split-K slices per GEMM
 
 struct FusedArgs {
     const __nv_bfloat16* x;       // [T, H]
-    const int32_t* permuted_rows; // [R]
-    const Tile* tiles;
-    const int32_t* num_tiles;
-    const float* topk_weights;    // [R]
+    const float* logits;          // [T, E]
+    int32_t* ids_out;             // [R]     routing outputs, written by CTA 0
+    float* weights_out;           // [R]
+    int32_t* offsets_out;         // [E + 1]
+    int32_t* rows_out;            // [R]
     __nv_bfloat16* act;           // [I / 64, R, 64] (K-blocked)
     float* part2;                 // [S2, R, H] when the w2 split is > 1
     __nv_bfloat16* y;             // [R, H] when the w2 split is 1
     __nv_bfloat16* out;           // [T, H]
-    int32_t* tile_ready;          // [max_tiles] w13 arrivals, zero at entry
-    int32_t* token_ready;         // [T * fb2] w2 row arrivals, zero at entry
-    int32_t* w2_next;             // w2 units handed out at run time, zero at entry
+    int32_t* tile_ready;          // [max_tiles] w13 arrivals
+    int32_t* token_ready;         // [T * fb2] w2 row arrivals
+    int32_t* w2_next;             // w2 units handed out at run time
+    int n_counters;               // the three above, contiguous: zeroed by CTA 0 every call
+    unsigned long long* ready;    // = gen once CTA 0 has zeroed them
+    unsigned long long gen;       // unique to this call
     int32_t* split_out;           // [2] 1, S2 (CTA 0)
     int32_t* err;
     const float* s13;             // W8: [E, 2I] w13 row scales
     const float* s2;              // W8: [E, H] w2 row scales
-    int k, H, I, R;
+    int T, E, k, H, I, R;
     int kt13, kt2;                // K tiles: H / 64, I / 64
     int fb13, fb2;                // I / 128 gate/up block pairs; ceil(H / 256) w2 block pairs
     int s2_max;
@@ -122,6 +127,25 @@ struct ComboScratch {
     float w[kMaxK];
 };
 
+// The routing every CTA does for itself (one-launch FFN: at most 64 tokens, so at
+// most 1024 expanded rows, and at most 1024 experts): permuted rows, routing
+// weights by expanded row, expert offsets, and the expert of each tile (every
+// expert's rows fit one tile, so tile j is the j-th touched expert).  After the
+// unit table in shared memory.
+constexpr int kMaxRows = kMaxK * 64;
+constexpr int kMaxExperts = 1024;
+struct alignas(16) RouteSmem {
+    int16_t rows[kMaxRows];
+    int16_t tile_expert[kMaxExperts];
+    int16_t off[kMaxExperts + 8];
+    float w[kMaxRows];
+    int n_tiles;
+};
+constexpr int kFusedReserve = kUnitTableBytes + (int)sizeof(RouteSmem);
+
+template <int NT>
+using FCfg = Cfg<0, NT, kFusedReserve>;
+
 // The FP8-weight kernel's buffers.  Shared memory after the 1 KB alignment
 // slack: B (kSB token tiles), then A8 (kS8 pair stages: two [128 x 128]-byte
 // E4M3 boxes in the 128-byte swizzle, K tiles kt and kt + 1, written by TMA);
@@ -134,7 +158,7 @@ struct ComboScratch {
 // A8, A, B.
 template <int NT>
 struct W8Cfg {
-    using C = Cfg<0, NT>;
+    using C = FCfg<NT>;
     static constexpr int kA8Bytes = 2 * kBM * 2 * kBK;
     static constexpr int kBoxBytes = kBM * 2 * kBK;  // one [128 x 128]-byte box
     static constexpr int kBBytes = C::kBTileBytes;
@@ -149,7 +173,7 @@ struct W8Cfg {
     // four of these M = 128, N <= 64 MMAs cost), so both rings have even depth
     // and their "empty" barriers are per slot pair.
     static_assert(kSA % 2 == 0 && kSB % 2 == 0, "slot pairs");
-    static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kUnitTableBytes;
+    static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kFusedReserve;
     static constexpr int kS8Raw = (C::kMaxSmem - kFixed - kSB * kBBytes) / kA8Bytes;
     static constexpr int kS8 = kS8Raw < 16 - kSA - kSB ? kS8Raw : 16 - kSA - kSB;
     static constexpr int kRingBytes = kSB * kBBytes + kS8 * kA8Bytes;
@@ -210,6 +234,158 @@ __device__ __forceinline__ bool warp_wait_count(const int32_t* ctr, int target,
     }
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Bounded wait until CTA 0 has zeroed this call's arrival counters (*ready ==
+// gen, read with acquire).  False on a timeout, a local abort or another CTA's
+// recorded error.
+__device__ __forceinline__ bool wait_counters(const FusedArgs& a, volatile int* abort)
+{
+    if (ld_acquire_gpu_u64(a.ready) == a.gen) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        __nanosleep(64);
+        if (ld_acquire_gpu_u64(a.ready) == a.gen) return true;
+        if (*abort || *reinterpret_cast<const volatile int32_t*>(a.err) == kDeviceErrorMagic ||
+            globaltimer_ns() - t0 > 2000000000ull)
+            return false;
+    }
+}
+
+// Routes the T tokens in this CTA (every thread calls; ends with a barrier).
+// scratch: shared memory unused until the producer starts, at least
+// route_scratch_bytes(warps) bytes.  Per token one warp stages its E logits in
+// shared memory, then takes the k experts in k rounds of warp arg-max over the
+// experts not yet taken (larger logit first, then the lower expert: the order of
+// the routing kernels), lane j keeping the j-th; the weights are those kernels'
+// softmax, bit for bit.  Then per-expert counts, offsets (a block scan), the
+// tiles (touched experts in order) and the stable permutation (one warp, rows in
+// ascending order, ranks from peer masks).  CTA 0 also writes the user-visible
+// routing outputs.
+constexpr int route_scratch_bytes(int warps)
+{
+    return warps * kMaxExperts * 4 + (kMaxExperts + kMaxRows + 32) * 4;
+}
+
+__device__ __forceinline__ void route_tokens(const FusedArgs& a, RouteSmem* rs, uint8_t* scratch)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    float* myrow = reinterpret_cast<float*>(scratch) + warp * kMaxExperts;
+    int* cnt = reinterpret_cast<int*>(scratch) + nwarps * kMaxExperts;  // [E], later cursors
+    int* ids_s = cnt + kMaxExperts;                                     // [R]
+    int* sums = ids_s + kMaxRows;                                       // [32]
+    const int E = a.E, k = a.k;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const int M = (E + 31) / 32;
+    for (int t = warp; t < a.T; t += nwarps) {
+        const float* src = a.logits + (size_t)t * E;
+        for (int e = lane; e < E; e += 32) myrow[e] = __ldg(src + e);
+        __syncwarp();
+        uint32_t taken = 0;  // bit m: expert 32 m + lane already selected
+        float my_l = -INFINITY;
+        int my_e = 0;
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int be = kNoIndex;
+            for (int m = 0; m < M; ++m) {  // experts ascend, so '>' keeps the lower one
+                const int e = m * 32 + lane;
+                if (e < E && !((taken >> m) & 1u)) {
+                    const float v = myrow[e];
+                    if (be == kNoIndex || v > bv) {
+                        bv = v;
+                        be = e;
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, bv, off);
+                const int oi = __shfl_xor_sync(kFull, be, off);
+                if (key_before(ov, oi, bv, be)) {
+                    bv = ov;
+                    be = oi;
+                }
+            }
+            if (lane == j) {
+                my_l = bv;
+                my_e = be;
+            }
+            if (be != kNoIndex && (be & 31) == lane) taken |= 1u << (be >> 5);
+        }
+        const float w = softmax_weight(my_l, k, lane);
+        if (lane < k) {
+            const int r = t * k + lane;
+            ids_s[r] = my_e;
+            rs->w[r] = w;
+            atomicAdd(&cnt[my_e], 1);
+            if (blockIdx.x == 0) {
+                a.ids_out[r] = my_e;
+                a.weights_out[r] = w;
+            }
+        }
+        __syncwarp();  // myrow is rewritten for the warp's next token
+    }
+    __syncthreads();
+    // offsets and tiles: thread i owns experts 2 i and 2 i + 1 (blockDim >= E / 2)
+    const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+    const int c0 = e0 < E ? cnt[e0] : 0, c1 = e1 < E ? cnt[e1] : 0;
+    int total, ntiles;
+    const int base = block_exclusive_scan(c0 + c1, sums, total);
+    const int tbase = block_exclusive_scan((c0 > 0) + (c1 > 0), sums, ntiles);
+    if (e0 < E) {
+        rs->off[e0] = (int16_t)base;
+        cnt[e0] = base;  // the cursor of the stable scatter
+        if (c0) rs->tile_expert[tbase] = (int16_t)e0;
+        if (blockIdx.x == 0) a.offsets_out[e0] = base;
+    }
+    if (e1 < E) {
+        rs->off[e1] = (int16_t)(base + c0);
+        cnt[e1] = base + c0;
+        if (c1) rs->tile_expert[tbase + (c0 > 0)] = (int16_t)e1;
+        if (blockIdx.x == 0) a.offsets_out[e1] = base + c0;
+    }
+    if (threadIdx.x == 0) {
+        rs->off[E] = (int16_t)total;
+        rs->n_tiles = ntiles;
+        if (blockIdx.x == 0) a.offsets_out[E] = total;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned lt = (1u << lane) - 1u;
+        for (int r0 = 0; r0 < a.R; r0 += 32) {
+            const int r = r0 + lane;
+            const bool valid = r < a.R;
+            const int e = valid ? ids_s[r] : -1;
+            const unsigned vm = __ballot_sync(kFull, valid);
+            unsigned peers = 0;
+            int pos = 0;
+            if (valid) {
+                peers = __match_any_sync(vm, e);
+                pos = cnt[e] + __popc(peers & lt);
+            }
+            __syncwarp();
+            if (valid) {
+                rs->rows[pos] = (int16_t)r;
+                if (blockIdx.x == 0) a.rows_out[pos] = r;
+                if (lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+}
+
 // W8: tm_w13 / tm_w2 map E4M3 codes ([128 x 128]-byte boxes, 128-byte swizzle).
 template <int NT, bool W8>
 __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
@@ -217,7 +393,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_w2,
                      const __grid_constant__ CUtensorMap tm_act, const FusedArgs a)
 {
-    using C = Cfg<0, NT>;
+    using C = FCfg<NT>;
     using R8 = W8Cfg<NT>;
     static_assert(NT <= 64, "weight-streaming tiles");
     extern __shared__ uint8_t smem_raw[];
@@ -234,6 +410,9 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     int* tok_off = reinterpret_cast<int*>(combo + 1);
     int4* unit_tab = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(aux) + C::kAuxBytes);
     int* tab_seq = reinterpret_cast<int*>(unit_tab + 2 * kUnitTable);
+    RouteSmem* rs = reinterpret_cast<RouteSmem*>(tab_seq + kUnitTable);
+    static_assert(route_scratch_bytes((W8 ? R8::kThreads : kThreads) / 32) <= kRingBytes,
+                  "routing scratch");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -279,12 +458,24 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = aux->tmem_base;
 
-    // the tile list, permuted rows, routing weights and zeroed counters come from
-    // the permutation kernel right before
+    // the inputs, and the workspace, once whatever ran before on the stream is done
     pdl_wait();
     pdl_launch_dependents();
+    volatile int* abort_flag = &aux->abort;
+    // CTA 0 zeroes the arrival counters and publishes this call's generation; every
+    // role waits for it (wait_counters) before its first counter access, which
+    // comes after at least one unit of work
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < a.n_counters; i += blockDim.x) a.tile_ready[i] = 0;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            st_release_gpu_u64(a.ready, a.gen);
+        }
+    }
+    route_tokens(a, rs, ring);  // the ring is free until the producer's first load
 
-    const int ntiles = __ldcg(a.num_tiles);
+    const int ntiles = rs->n_tiles;
     // w13 is not split here: its epilogue writes bf16 act directly, which each w2
     // stage then loads with one TMA.  w2 is split only as far as ~4 waves of units
     // need: the run-time hand-out already balances the tail, and every extra
@@ -302,7 +493,6 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         a.split_out[0] = 1;
         a.split_out[1] = S2;
     }
-    volatile int* abort_flag = &aux->abort;
 
     // Schedule.  CTA b first runs w13 units b, b + G, ...  When U13 is not a
     // multiple of G, the CTAs with one unit fewer ("light", b >= U13 % G) next
@@ -334,16 +524,14 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         const int ktps = un.ph ? ktps2 : a.kt13, nkt = un.ph ? a.kt2 : a.kt13;
         un.split = v % S;
         const int rest = v / S;
-        const Tile probe = load_tile(a.tiles + rest / fbc);
-        const int local = rest - fbc * probe.first;
-        un.fb = local / probe.count;
-        un.tile = probe.first + local % probe.count;
+        // one tile per expert: tile-major, feature block minor
+        un.tile = rest / fbc;
+        un.fb = rest % fbc;
         un.kt0 = un.split * ktps;
         un.kt1 = min(nkt, un.kt0 + ktps);
-        const Tile t = load_tile(a.tiles + un.tile);
-        un.expert = t.expert;
-        un.row_start = t.row_start;
-        un.rows = t.rows;
+        un.expert = rs->tile_expert[un.tile];
+        un.row_start = rs->off[un.expert];
+        un.rows = rs->off[un.expert + 1] - un.row_start;
         return un;
     };
     auto put = [&](int slot, const Unit& un) {
@@ -408,11 +596,16 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             int issued[16];
             for (int s = 0; s < NS; ++s) issued[s] = 0;
             bool ok = true;
+            bool counters = false;  // this call's counters are zeroed (wait_counters)
             for (int i = 0; ok; ++i) {
                 Unit un;
                 if (i < n_static) {
                     un = get(i);
                 } else {  // claim the next w2 unit and publish it to the other roles
+                    if (!counters && !(counters = wait_counters(a, abort_flag))) {
+                        flag_error(a.err, aux);
+                        break;
+                    }
                     const int v = rest0 + atomicAdd(a.w2_next, 1);
                     if (v < U2) {
                         un = decode(U13 + v);
@@ -571,13 +764,16 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         int last_tma[R8::kSB];  // stage of each slot's latest use when that was a TMA, else -1
         for (int sb = 0; sb < R8::kSB; ++sb) last_tma[sb] = -1;
         bool ok = true;
+        bool counters = false;
         for (int i = 0; ok; ++i) {
             const Unit un = get(i);
             if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
             const Unit& t = un;
             if (un.ph == 1 && un.tile != ready_tile) {
                 // every w13 unit of this tile has stored its act rows
-                if (!warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
+                if ((!counters &&
+                     !(counters = __all_sync(0xffffffffu, wait_counters(a, abort_flag)))) ||
+                    !warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
                     if (lane == 0) flag_error(a.err, aux);
                     ok = false;
                     break;
@@ -589,7 +785,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 __syncwarp();  // earlier copies' addresses are all issued
                 if (un.ph == 0)
                     for (int j = lane; j < t.rows; j += 32)
-                        my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
+                        my_off[j] = (rs->rows[t.row_start + j] / a.k) * a.H;
                 __syncwarp();
                 cur_tile = un.tile;
                 cur_ph = un.ph;
@@ -703,6 +899,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             int q = 0;  // global stage sequence number (same as the producer's)
             int cur_tile = -1, cur_ph = -1, ready_tile = -1;
             bool ok = true;
+            bool counters = false;
             for (int i = 0; ok; ++i) {
                 const Unit un = get(i);
                 if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
@@ -714,7 +911,9 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 const Unit& t = un;
                 if (un.ph == 1 && un.tile != ready_tile) {
                     // every w13 unit of this tile has stored its act rows or slices
-                    if (!warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
+                    if ((!counters &&
+                         !(counters = __all_sync(0xffffffffu, wait_counters(a, abort_flag)))) ||
+                        !warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
                         if (lane == 0) flag_error(a.err, aux);
                         ok = false;
                         break;
@@ -726,7 +925,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                     __syncwarp();  // earlier copies' addresses are all issued
                     if (un.ph == 0)
                         for (int j = lane; j < t.rows; j += 32)
-                            my_off[j] = (a.permuted_rows[t.row_start + j] / a.k) * a.H;
+                            my_off[j] = (rs->rows[t.row_start + j] / a.k) * a.H;
                     __syncwarp();
                     cur_tile = un.tile;
                     cur_ph = un.ph;
@@ -783,7 +982,12 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         const int f_local = qw * 32 + lane;       // feature inside the 128-row block
         uint8_t* gstage = staging + grp * 2 * (kStageRows * kStageRowBytes);
         int chunk = 0;  // staging chunks issued by this group (buffer parity)
-        for (int lu = 0;; ++lu) {
+        // every epilogue thread publishes to (or waits on) the counters: before its
+        // first unit's accumulator is even ready, CTA 0 has long zeroed them (the
+        // outcome is made the same in all four warps of the group)
+        const bool counters = !named_bar_or(1 + grp, 128, !wait_counters(a, abort_flag));
+        if (!counters) flag_error(a.err, aux);
+        for (int lu = 0; counters; ++lu) {
             const Unit un = get(lu);
             const Unit& t = un;
             const int b = lu % NBUF;
@@ -867,7 +1071,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                         // act: K block 2 fb + c / 8 of row p; y: expanded-id row
                         __nv_bfloat16* dst = ph == 0
                             ? a.act + ((size_t)(2 * un.fb + (c >> 3)) * a.R + p) * kBK + (c & 7) * 8
-                            : a.y + (size_t)a.permuted_rows[p] * a.H + un.fb * 2 * kBM + c * 8;
+                            : a.y + (size_t)rs->rows[p] * a.H + un.fb * 2 * kBM + c * 8;
                         *reinterpret_cast<uint4*>(dst) = val;
                     }
                     ++chunk;
@@ -885,7 +1089,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                         if (j >= jend) break;
                         const int p = t.row_start + j;
                         {  // w2 slice: fp32 by expanded id
-                            const int r = a.permuted_rows[p];
+                            const int r = rs->rows[p];
                             float* prow = a.part2 + ((size_t)un.split * a.R + r) * a.H;
                             float g0 = __uint_as_float(gv[jj]), g1 = __uint_as_float(vv[jj]);
                             if constexpr (W8) {
@@ -909,7 +1113,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             if (ph == 0) {
                 if (gt == 0) red_release_gpu_add(a.tile_ready + un.tile, 1);
             } else if (gt < jend - jbeg) {
-                const int tok = a.permuted_rows[t.row_start + jbeg + gt] / a.k;
+                const int tok = rs->rows[t.row_start + jbeg + gt] / a.k;
                 red_release_gpu_add(a.token_ready + (size_t)tok * a.fb2 + un.fb, 1);
             }
         }
@@ -926,7 +1130,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             if (warp == kEpiWarp0) {
                 ready = warp_wait_count(a.token_ready + task, token_target, abort_flag, a.err);
                 if (!ready && lane == 0) flag_error(a.err, aux);
-                if (ready && lane < a.k) combo->w[lane] = a.topk_weights[(size_t)tok * a.k + lane];
+                if (ready && lane < a.k) combo->w[lane] = rs->w[tok * a.k + lane];
             }
             if (named_bar_or(3, 256, !ready || *abort_flag)) break;  // uniform over the 8 warps
             const int c0 = fb * 2 * kBM;
@@ -992,12 +1196,12 @@ template <int NT, bool W8>
 cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const CUtensorMap& ta,
                             const FusedArgs& a, int grid, cudaStream_t st)
 {
-    using C = Cfg<0, NT>;
+    using C = FCfg<NT>;
     // the combine's weights sit in the slack Cfg reserves next to Aux; the unit
-    // table follows the aux area
+    // table and the routing tables follow the aux area
     static_assert(sizeof(Aux) + sizeof(ComboScratch) <= 1024, "aux area");
-    static_assert(C::kAuxBytes % 16 == 0, "unit table alignment");
-    constexpr int smem = W8 ? W8Cfg<NT>::kSmemBytes : C::kSmemBytes + kUnitTableBytes;
+    static_assert(C::kAuxBytes % 16 == 0 && kUnitTableBytes % 16 == 0, "table alignment");
+    constexpr int smem = W8 ? W8Cfg<NT>::kSmemBytes : C::kSmemBytes + kFusedReserve;
     static_assert(smem <= C::kMaxSmem, "shared memory");
     auto kern = fused_ffn_kernel<NT, W8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1010,10 +1214,11 @@ cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const
 
 bool fused_ffn_eligible(int T, int E, int k, int H, int I, const FfnPlan& plan)
 {
-    (void)E;
     (void)H;
     (void)I;
-    return plan.nt <= 64 && (long)T * k <= kSmallRows && k <= kMaxK && plan.s2_max <= kMaxSplits;
+    // every expert's rows in one tile (plan.nt >= T), and the routing tables fit
+    return plan.nt <= 64 && plan.nt >= T && (long)T * k <= kMaxRows && k <= kMaxK &&
+           E <= kMaxExperts && plan.s2_max <= kMaxSplits;
 }
 
 int fused_ffn_counters(int T, int H, const FfnPlan& plan)
@@ -1039,10 +1244,11 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     if (err != cudaSuccess) return err;
     FusedArgs a = {};
     a.x = static_cast<const __nv_bfloat16*>(b.x);
-    a.permuted_rows = b.permuted_rows;
-    a.tiles = b.tiles;
-    a.num_tiles = b.num_tiles;
-    a.topk_weights = b.topk_weights;
+    a.logits = b.logits;
+    a.ids_out = b.topk_ids;
+    a.weights_out = b.topk_weights;
+    a.offsets_out = b.expert_offsets;
+    a.rows_out = b.permuted_rows;
     a.act = static_cast<__nv_bfloat16*>(b.act);
     a.part2 = b.part2;
     a.y = static_cast<__nv_bfloat16*>(b.y);
@@ -1050,8 +1256,13 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     a.tile_ready = b.counters;
     a.token_ready = b.counters + plan.max_tiles;
     a.w2_next = a.token_ready + (size_t)T * ((H / kBM + 1) / 2);
+    a.n_counters = fused_ffn_counters(T, H, plan);
+    a.ready = b.ready;
+    a.gen = b.gen;
     a.split_out = b.splits;
     a.err = b.err;
+    a.T = T;
+    a.E = E;
     a.k = k;
     a.H = H;
     a.I = I;

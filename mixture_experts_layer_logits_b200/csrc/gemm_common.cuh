@@ -30,8 +30,9 @@ constexpr int kStageRowBytes = 512;  // one token row: 256 bf16 outputs
 constexpr int kATileBytes = kBM * kBK * 2;
 
 // Shared-memory ring of one CTA.  MODE 0: the B operand (token rows) is written by
-// the gather warps; MODE 1: it is loaded by TMA with the weights.
-template <int MODE, int NT>
+// the gather warps; MODE 1: it is loaded by TMA with the weights.  RESERVE bytes
+// after the aux area are left for the kernel's own tables.
+template <int MODE, int NT, int RESERVE = 0>
 struct Cfg {
     static constexpr int kNA = 2;                                  // A tiles per stage
     static constexpr int kBTileBytes = NT * kBK * 2;
@@ -41,7 +42,7 @@ struct Cfg {
     static constexpr int kAuxBytes = 1024 + kGatherWarps * NT * 4;
     static constexpr int kStagingBytes = 2 * 2 * kStageRows * kStageRowBytes;  // 2 groups x 2 bufs
     static constexpr int kStagesRaw =
-        (kMaxSmem - 1024 - kAuxBytes - kStagingBytes) / kStageBytes;
+        (kMaxSmem - 1024 - kAuxBytes - kStagingBytes - RESERVE) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kAccCols = 2 * NT;                        // per accumulator buffer
     static constexpr int kNBufRaw = 512 / kAccCols;                // accumulators in flight

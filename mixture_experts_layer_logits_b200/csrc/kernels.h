@@ -56,19 +56,9 @@ struct PermuteAux {
     Tile* tiles;           // [max_tiles]
     int32_t* num_tiles;    // device scalar
     int nt;                // token rows per tile (the GEMM's N tile)
-    int32_t* counters;     // split-K arrival counters to zero, [n_counters]
-    int n_counters;
     int32_t* chunk_counts; // [n_chunks + 1, E] scratch of the multi-CTA path
     int32_t* err;          // the error word (debug-build index checks); may be null
     int max_tiles;         // entries of `tiles`
-    // L2 prefetch of w13 for the one-launch FFN (single-CTA path, with routing):
-    // the launch gets pf_units CTAs, and CTA b >= 1 prefetches the first pf_kt K
-    // tiles of the gate and up blocks of w13 unit b (fused CTA b's first unit)
-    // through the tensor map passed with the launch.  pf_units = 0: off.
-    int pf_units;
-    int pf_fb13;   // I / 128
-    int pf_I;
-    int pf_kt;
 };
 
 // Records the cudaError_t that moe_last_cuda_error() reports on this host thread.
@@ -110,8 +100,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids,
 constexpr int kSmallRows = 4096;
 cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k, int32_t* ids,
                                        float* weights, int32_t* offsets, int32_t* rows,
-                                       const PermuteAux& aux, cudaStream_t st,
-                                       const CUtensorMap* pf_w13 = nullptr);
+                                       const PermuteAux& aux, cudaStream_t st);
 
 // Multi-CTA path: per-chunk counts, per-expert prefixes over the chunks (and the
 // expert totals), then a per-chunk stable scatter (CTA 0 also writes offsets and
@@ -155,23 +144,29 @@ cudaError_t launch_grouped_ffn(const FfnBuffers& b, int T, int E, int k, int H, 
                                const FfnPlan& plan, cudaStream_t st,
                                cudaEvent_t between_gemms = nullptr, bool reduce_y = true);
 
-// w13 + SwiGLU, w2 and the combine in one persistent launch (fused_ffn.cu), for
-// weight-streaming shapes: at most 64 tokens, so every expert's rows fit one tile.
+// Routing, the permutation, w13 + SwiGLU, w2 and the combine in one persistent
+// launch (fused_ffn.cu), for weight-streaming shapes: at most 64 tokens, so every
+// expert's rows fit one tile.  Every CTA routes the tokens itself; CTA 0 writes
+// the routing outputs and zeroes the arrival counters of this call, then sets
+// *ready = gen (a value unique to the call) for the others.
 struct FusedBuffers {
     const void* x;
+    const float* logits;
     const void* w13;   // bf16 weights, or E4M3 codes when s13 is set
     const void* w2;
     const float* s13;  // E4M3 weights: [E, 2I] and [E, H] fp32 row scales; else nullptr
     const float* s2;
-    const int32_t* permuted_rows;
-    const Tile* tiles;
-    const int32_t* num_tiles;
-    const float* topk_weights;
+    int32_t* topk_ids;        // routing outputs [R], [R], [E + 1], [R]
+    float* topk_weights;
+    int32_t* expert_offsets;
+    int32_t* permuted_rows;
     void* act;         // bf16 [I / 64, R, 64] (K-blocked)
     float* part2;      // fp32 [s2_max, R, H]
     void* y;           // bf16 [R, H]
     void* out;         // bf16 [T, H]
-    int32_t* counters; // [fused_ffn_counters()], zeroed by the permutation kernel
+    int32_t* counters; // [fused_ffn_counters()]
+    unsigned long long* ready;
+    unsigned long long gen;
     int32_t* splits;   // [2]
     int32_t* err;
 };

@@ -8,6 +8,10 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+#include <chrono>
+#include <random>
+
 #include "gemm_common.cuh"
 #include "kernels.h"
 #include "moe.h"
@@ -76,11 +80,11 @@ bool combine_shape_ok(const moe_shape_t& s)
 
 struct Layout {
     size_t err, ids, weights, offsets, rows, tiles, num_tiles, splits, chunks, partials, act, y,
-        partials2, counters, total;
+        partials2, counters, ready, total;
     FfnPlan plan;
     bool ffn;
     bool fused;      // the shape qualifies for the one-launch FFN + combine
-    int n_counters;  // its arrival counters (zeroed by the permutation kernel)
+    int n_counters;  // its arrival counters (zeroed by its own CTA 0 every call)
 };
 
 Layout layout_for(const moe_shape_t& s)
@@ -120,6 +124,7 @@ Layout layout_for(const moe_shape_t& s)
             L.partials2 = take(p2 * sizeof(float));
             L.n_counters = fused_ffn_counters(s.T, H, L.plan);
             L.counters = take((size_t)L.n_counters * sizeof(int32_t));
+            L.ready = take(sizeof(unsigned long long));
         }
     }
     L.total = off;
@@ -159,59 +164,43 @@ PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
     a.tiles = at<Tile>(ws, L.tiles);
     a.num_tiles = at<int32_t>(ws, L.num_tiles);
     a.nt = L.plan.nt;
-    a.counters = L.fused ? at<int32_t>(ws, L.counters) : nullptr;
-    a.n_counters = L.fused ? L.n_counters : 0;
     a.chunk_counts = at<int32_t>(ws, L.chunks);
     a.err = at<int32_t>(ws, L.err);
     a.max_tiles = L.plan.max_tiles;
-    a.pf_units = 0;
-    a.pf_fb13 = a.pf_I = a.pf_kt = 0;
     (void)s;
     return a;
 }
 
-// w13_prefetch: for the one-launch FFN, the w13 weights (bf16, or E4M3 codes when
-// prefetch_e4m3) whose first K tiles the permutation kernel prefetches into L2
-// (single-CTA path only).
 moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, const moe_shape_t& s,
                          int32_t* offsets, int32_t* rows, void* ws, const Layout& L,
-                         cudaStream_t st, const void* w13_prefetch = nullptr,
-                         bool prefetch_e4m3 = false)
+                         cudaStream_t st)
 {
     PermuteAux aux = make_aux(ws, L, s);
     const long R = (long)s.T * s.top_k;
     cudaError_t e;
     if (R <= kSmallRows) {
-        CUtensorMap pf;
-        const CUtensorMap* pf_map = nullptr;
-        const uint64_t pf_rows = (uint64_t)s.E * 2 * s.I;
-        if (w13_prefetch &&
-            (prefetch_e4m3
-                 ? gemm::make_tmap_u8(&pf, w13_prefetch, pf_rows, (uint64_t)s.H, gemm::kBM)
-                 : gemm::make_tmap(&pf, w13_prefetch, pf_rows, (uint64_t)s.H, gemm::kBM)) ==
-                cudaSuccess) {
-            pf_map = &pf;
-            // each fused CTA's first w13 unit, as far as there can be w13 units:
-            // at most min(E, T*k) tiles (one per touched expert), I/128 units each
-            const long max_units13 = (long)(s.E < R ? s.E : R) * (s.I / gemm::kBM);
-            aux.pf_units = (int)(max_units13 < device_sms() ? max_units13 : device_sms());
-            aux.pf_fb13 = s.I / gemm::kBM;
-            aux.pf_I = s.I;
-            // 16 K tiles (2 x 128 x 1024 weights per CTA) cover the routing and
-            // fused-kernel set-up window; 8 left HBM idle part of it, 20 and 24
-            // gained nothing more (same-B200 A/B)
-            // (E4M3 codes: the same bytes are twice the K tiles)
-            const int kPrefetchKt = prefetch_e4m3 ? 32 : 16;
-            aux.pf_kt = s.H / gemm::kBK < kPrefetchKt ? s.H / gemm::kBK : kPrefetchKt;
-        }
         e = launch_small_route_permute(logits, s.T, s.E, s.top_k, ids, weights, offsets, rows, aux,
-                                       st, pf_map);
+                                       st);
     } else {
         e = cudaSuccess;
         if (logits) e = launch_route(logits, s.T, s.E, s.top_k, ids, weights, st);
         if (e == cudaSuccess) e = launch_large_permute(ids, s.T, s.E, s.top_k, offsets, rows, aux, st);
     }
     return cuda_status(e);
+}
+
+// A value unique to each one-launch FFN call (the generation its CTA 0 publishes
+// once the call's counters are zeroed): a per-process random start plus a
+// counter, so that neither an earlier call's value nor stale workspace bytes
+// match it.
+unsigned long long next_generation()
+{
+    static std::atomic<unsigned long long> counter{[] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 32) ^ rd() ^
+               (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    }()};
+    return counter.fetch_add(0x9E3779B97F4A7C15ull) + 0x9E3779B97F4A7C15ull;
 }
 
 moe_status_t run_ffn(const void* x, const void* w13, const void* w2, const int32_t* rows,
@@ -343,27 +332,29 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
     if (w8 && !L.fused) return MOE_ERR_UNSUPPORTED_SHAPE;
     const bool fused = w8 || (L.fused && fused_enabled());
     moe_status_t r = mark(0);
-    if (r == MOE_OK)
-        r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st, fused ? w13 : nullptr, w8);
-    if (r == MOE_OK) r = mark(1);
     if (fused) {
-        // one launch: w13, w2 and the combine (the stage events in between all
-        // mark its end)
+        // one launch: routing and the permutation (inside every CTA), w13, w2 and
+        // the combine; events [1] .. [4] all mark its end except [1], recorded
+        // right after [0]
+        if (r == MOE_OK) r = mark(1);
         FusedBuffers b;
         b.x = x;
+        b.logits = logits;
         b.w13 = w13;
         b.w2 = w2;
         b.s13 = s13;
         b.s2 = s2;
-        b.permuted_rows = rows;
-        b.tiles = at<Tile>(ws, L.tiles);
-        b.num_tiles = at<int32_t>(ws, L.num_tiles);
+        b.topk_ids = ids;
         b.topk_weights = wts;
+        b.expert_offsets = offs;
+        b.permuted_rows = rows;
         b.act = at<void>(ws, L.act);
         b.part2 = at<float>(ws, L.partials2);
         b.y = y;
         b.out = out;
         b.counters = at<int32_t>(ws, L.counters);
+        b.ready = at<unsigned long long>(ws, L.ready);
+        b.gen = next_generation();
         b.splits = at<int32_t>(ws, L.splits);
         b.err = at<int32_t>(ws, L.err);
         FfnPlan plan = L.plan;
@@ -373,6 +364,8 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
         for (int i = 2; i <= 4 && r == MOE_OK; ++i) r = mark(i);
         return r;
     }
+    if (r == MOE_OK) r = run_permute(logits, ids, wts, s, offs, rows, ws, L, st);
+    if (r == MOE_OK) r = mark(1);
     // a split w2 is reduced inside the combine (one launch fewer)
     const bool split2 = L.plan.s2_max > 1;
     if (r == MOE_OK)
@@ -445,9 +438,10 @@ int moe_forward_kernel_count(moe_shape_t s)
     if (!ffn_shape_ok(s)) return 0;
     const long R = (long)s.T * s.top_k;
     const Layout L = layout_for(s);
-    // routing and permutation: one kernel, or route + count + scan + scatter
+    // the one-launch FFN routes and permutes inside its own launch
+    if (L.fused && fused_enabled()) return 1;
+    // routing and permutation: one kernel, or route + count + prefix + scatter
     const int route_permute = R <= kSmallRows ? 1 : 4;
-    if (L.fused && fused_enabled()) return route_permute + 1;
     // w13, [SwiGLU finalize], w2, combine
     return route_permute + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
 }

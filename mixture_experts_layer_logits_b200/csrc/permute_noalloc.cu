@@ -80,9 +80,6 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t
         aux.err = reinterpret_cast<int32_t*>(p + kCountBytes + kTileBytes + 16);
         aux.nt = 1 << 30;  // one tile per expert: the tile list stays within 1024 entries
         aux.max_tiles = 1024;
-        aux.counters = nullptr;
-        aux.n_counters = 0;
-        aux.pf_units = aux.pf_fb13 = aux.pf_I = aux.pf_kt = 0;
         cudaStream_t st = static_cast<cudaStream_t>(stream);
         int32_t* ids = const_cast<int32_t*>(topk_ids);
         if (R <= kSmallRows)

@@ -22,19 +22,12 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+#include "route_common.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kNoIndex = 0x7fffffff;
-
-// (va, ia) ranks before (vb, ib)?
-__device__ __forceinline__ bool key_before(float va, int ia, float vb, int ib)
-{
-    return va > vb || (va == vb && ia < ib);
-}
 
 // Sorts one (value, index) key per lane across groups of W lanes (W = 16: each
 // half-warp on its own; W = 32: the warp) so that the group's first lane holds
@@ -165,28 +158,6 @@ __device__ __forceinline__ void sort_candidates(int total, int lane, const float
         warp_sort_keys<32>(cv, ci, lane);
     my_l = cv;
     my_id = ci;
-}
-
-// Softmax over the selected logits (lane j holds the j-th; l_0 is the largest)
-// and the outputs.  The sum is a fixed xor-tree over lanes 0..15 (lanes >= k
-// contribute 0), so it is deterministic.
-__device__ __forceinline__ void write_selection(float my_l, int my_id, int k, int lane,
-                                                int32_t* __restrict__ ids,
-                                                float* __restrict__ weights, int* ids_s)
-{
-    const float l0 = __shfl_sync(kFull, my_l, 0);
-    const float ex = (lane < k) ? expf(my_l - l0) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int off = 1; off < 16; off <<= 1) sum += __shfl_xor_sync(kFull, sum, off);
-    sum = __shfl_sync(kFull, sum, 0);
-    if (lane < k) {
-        if (ids) {
-            ids[lane] = my_id;
-            weights[lane] = ex / sum;
-        }
-        if (ids_s) ids_s[lane] = my_id;
-    }
 }
 
 // Exact selection when more than 32 experts reach the threshold (ties, -inf
@@ -347,40 +318,10 @@ __device__ __forceinline__ void warp_route_token(const float* __restrict__ row, 
     warp_select_token<V, VEC>(v, E, k, lane, ids, weights, ids_s, cand);
 }
 
-// Exclusive scan of one int per thread over the whole CTA (blockDim.x a
-// multiple of 32, <= 1024).  `sums` is shared scratch of 32 ints.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* sums, int& total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int n = __shfl_up_sync(kFull, incl, off);
-        if (lane >= off) incl += n;
-    }
-    if (lane == 31) sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int s = (lane < nw) ? sums[lane] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int n = __shfl_up_sync(kFull, s, off);
-            if (lane >= off) s += n;
-        }
-        sums[lane] = s;
-    }
-    __syncthreads();
-    const int prefix = (warp > 0) ? sums[warp - 1] : 0;
-    total = sums[nw - 1];
-    __syncthreads();
-    return prefix + incl - v;
-}
-
 // Thread e (< E) owns expert e with `count` rows at permuted offset `off` and
 // writes its tiles: as few as ceil(count / nt) allows, of near-equal size rounded
 // to the MMA's 16-column granule (so no tile is a short tail that streams a whole
 // weight block for a few rows), the last one taking the remainder.
-// Also zeroes the split-K counters.
 __device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int count, int off,
                                                       const PermuteAux& aux, int* sums)
 {
@@ -409,7 +350,6 @@ __device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int coun
         aux.tiles[start + i] = t;
     }
     if (threadIdx.x == 0) *aux.num_tiles = total;
-    for (int i = threadIdx.x; i < aux.n_counters; i += blockDim.x) aux.counters[i] = 0;
 }
 
 // Per-warp histogram of rows [r0, r1) of ids_s into table[warp*E + e].
@@ -540,52 +480,12 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 3)
 }
 
 // One CTA: (route) + count + scan + stable scatter + tile list, for T*k <= kSmallRows.
-// CTAs 1.. of the single-CTA permutation launch when the one-launch FFN follows
-// (aux.pf_units > 0).  Each routes the T tokens again (ids into shared memory
-// only; CTA 0 writes every output), ranks the touched experts -- with T no
-// larger than the tile height every expert's rows form one tile, so tile j is
-// the j-th touched expert -- and prefetches into L2 the first pf_kt K tiles of
-// the gate and up blocks of w13 unit blockIdx.x: the first unit of fused CTA
-// blockIdx.x (tile = unit / fb13, feature block = unit % fb13).  Spread over the
-// grid, the weight stream starts while CTA 0 is still permuting; from one SM
-// the prefetches would drain at a single TMA unit's rate.  A hint only.
-template <int V, bool VEC>
-__device__ __forceinline__ void prefetch_first_unit(const float* __restrict__ logits, int T, int E,
-                                                    int k, const PermuteAux& aux,
-                                                    const CUtensorMap* w13, int* flag,
-                                                    int (*sel)[16], float2 (*cand)[32], int* sums)
-{
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) flag[e] = 0;
-    __syncthreads();
-    for (int t = warp; t < T; t += 32) {
-        float v[V];
-        warp_load_row<V, VEC>(logits + (size_t)t * E, E, lane, v);
-        warp_select_token<V, VEC>(v, E, k, lane, nullptr, nullptr, sel[warp], cand[warp]);
-        __syncwarp();
-        if (lane < k) flag[sel[warp][lane]] = 1;
-        __syncwarp();
-    }
-    __syncthreads();
-    const int e = threadIdx.x;
-    const int touched = e < E ? flag[e] : 0;
-    int total;
-    const int rank = block_exclusive_scan(touched, sums, total);  // ends with a barrier
-    if (touched) flag[rank] = e;  // flag[j] = expert of tile j
-    __syncthreads();
-    const int tile = blockIdx.x / aux.pf_fb13, fb = blockIdx.x % aux.pf_fb13;
-    if (tile < total && threadIdx.x < 2 * aux.pf_kt) {
-        const int half = threadIdx.x / aux.pf_kt, kt = threadIdx.x % aux.pf_kt;
-        tma_prefetch_l2_2d(w13, kt * 64, flag[tile] * 2 * aux.pf_I + half * aux.pf_I + fb * 128);
-    }
-}
-
 template <int V, bool VEC>
 __global__ void __launch_bounds__(1024, 1)
     small_route_permute_kernel(const float* __restrict__ logits, int T, int E, int k,
                                int32_t* __restrict__ ids, float* __restrict__ weights,
                                int32_t* __restrict__ offsets, int32_t* __restrict__ rows_out,
-                               PermuteAux aux, const __grid_constant__ CUtensorMap pf_w13)
+                               PermuteAux aux)
 {
     extern __shared__ int smem[];
     __shared__ int sums[32];
@@ -598,11 +498,6 @@ __global__ void __launch_bounds__(1024, 1)
     pdl_wait();
     pdl_launch_dependents();
 
-    if (blockIdx.x > 0) {  // L2 prefetch CTAs (launched only with logits and aux.pf_units)
-        __shared__ int sel[32][16];
-        prefetch_first_unit<V, VEC>(logits, T, E, k, aux, &pf_w13, smem, sel, cand, sums);
-        return;
-    }
     if (logits) {
         // a warp's next token is loaded while its current one is selected
         float v[V];
@@ -843,34 +738,27 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* ids,
 template <int V, bool VEC>
 static cudaError_t launch_small_v(const float* logits, int T, int E, int k, int32_t* ids,
                                   float* weights, int32_t* offsets, int32_t* rows,
-                                  const PermuteAux& aux, cudaStream_t st, const CUtensorMap& pf)
+                                  const PermuteAux& aux, cudaStream_t st)
 {
     const int R = T * k;
     const size_t smem = sizeof(int) * (size_t)(((R + 3) & ~3) + 32 * E);  // >= E ints
     cudaError_t err = cudaFuncSetAttribute(small_route_permute_kernel<V, VEC>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int grid = (logits && aux.pf_units > 1) ? aux.pf_units : 1;  // CTAs 1.. prefetch
-    return launch(small_route_permute_kernel<V, VEC>, dim3(grid), dim3(1024), smem, st, logits, T,
-                  E, k, ids, weights, offsets, rows, aux, pf);
+    return launch(small_route_permute_kernel<V, VEC>, dim3(1), dim3(1024), smem, st, logits, T, E,
+                  k, ids, weights, offsets, rows, aux);
 }
 
 cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k, int32_t* ids,
                                        float* weights, int32_t* offsets, int32_t* rows,
-                                       const PermuteAux& aux, cudaStream_t st,
-                                       const CUtensorMap* pf_w13)
+                                       const PermuteAux& aux, cudaStream_t st)
 {
     const bool vec = (E % 4) == 0;
-    CUtensorMap none;
-    memset(&none, 0, sizeof(none));  // never read: pf_units == 0 without a map
-    PermuteAux a = aux;
-    if (!pf_w13) a.pf_units = 0;
-    const CUtensorMap& pf = pf_w13 ? *pf_w13 : none;
 #define MOE_SMALL(V)                                                                              \
     (vec && (V) >= 4 ? launch_small_v<V, ((V) >= 4)>(logits, T, E, k, ids, weights, offsets, rows, \
-                                                     a, st, pf)                                   \
-                     : launch_small_v<V, false>(logits, T, E, k, ids, weights, offsets, rows, a,   \
-                                                st, pf))
+                                                     aux, st)                                     \
+                     : launch_small_v<V, false>(logits, T, E, k, ids, weights, offsets, rows, aux, \
+                                                st))
     switch (logits ? values_per_lane(E) : 1) {
     case 1: return MOE_SMALL(1);
     case 2: return MOE_SMALL(2);

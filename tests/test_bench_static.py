@@ -46,7 +46,8 @@ def test_stage_work_counts_e4m3_weights_at_one_byte_plus_row_scales():
     bf = bench.stage_work(w, n)
     f8 = bench.stage_work(w, n, "e4m3")
     T, k, H, I = w.T, w.k, w.H, w.I
-    rest = T * H * 2 + T * k * 8 + T * H * 2  # x, routing weights and rows, out
+    # x, routing weights and rows, out; the routing's logits and outputs
+    rest = T * H * 2 + T * k * 8 + T * H * 2 + T * w.E * 4 + T * k * 12 + (w.E + 1) * 4
     assert bf["fused_ffn"]["bytes"] == n * 3 * I * H * 2 + rest
     assert f8["fused_ffn"]["bytes"] == n * (3 * I * H + (2 * I + H) * 4) + rest
     assert f8["fused_ffn"]["flops"] == bf["fused_ffn"]["flops"]  # same bf16 products

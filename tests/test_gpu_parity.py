@@ -274,6 +274,20 @@ def test_forward_without_pdl_is_identical(tmp_path):
     assert torch.equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("T,E,k", [(64, 8, 8), (40, 64, 16), (33, 1024, 16), (16, 1000, 5),
+                                   (2, 3, 3)])
+def test_fused_path_routing_adversarial(T, E, k):
+    """The one-launch path (T <= 64) routes inside its own kernel: all-equal rows,
+    signed zeros, -inf and ties at the k-th place give the oracle's ids bit for bit
+    and its weights, and the whole output matches the oracle."""
+    H, I = 128, 128
+    assert moe.moe_forward_fused(T, E, k, H, I)
+    w = wl.custom("adv", T, E, k, H, I)
+    d = inputs(w, seed=41)
+    d["logits"] = adversarial_logits(T, E, seed=T + E).cuda()
+    check_full(w, d)
+
+
 # Shapes for the one-launch FFN + combine (T <= 64): both w2 split choices,
 # the multi-launch path's w13 split both on (H >= 512) and off, an odd number
 # of 128-row w2 blocks, k = 16 over 1024 experts, one token, the largest routed
@@ -328,7 +342,7 @@ def test_fused_launch_against_multi_launch_and_oracle(tmp_path):
         w = _fused_workload(name, spec)
         d = wl.make_inputs(w, seed=13, device="cuda")
         assert moe.moe_forward_fused(w.T, w.E, w.k, w.H, w.I), name
-        assert moe.moe_forward_kernel_count(w.T, w.E, w.k, w.H, w.I) == 2, name
+        assert moe.moe_forward_kernel_count(w.T, w.E, w.k, w.H, w.I) == 1, name
         out, ids, wts, off, rows = run_forward(w, d)
         multi = ref[name]
         if w.H < 512:
