@@ -116,9 +116,11 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
  * x bf16 [T, H], logits fp32 [T, E], w13 bf16 [E, 2I, H], w2 bf16 [E, H, I]
  * -> out bf16 [T, H].  topk_ids, topk_weights, expert_offsets and permuted_rows
  * are optional outputs: pass NULL to keep them inside the workspace.
- * For weight-streaming shapes (T <= 64, see moe_forward_fused) w13, w2 and the
- * combine run as ONE persistent launch whose CTAs hand act rows and finished y
- * rows to each other through arrival counters in the workspace.  It sums w13
+ * For weight-streaming shapes (T <= 64, see moe_forward_fused) the whole layer
+ * runs as ONE persistent launch: every CTA routes and permutes the tokens itself
+ * (the same ids and, bit for bit, the same weights as moe_route), and the CTAs
+ * hand act rows and finished y rows to each other through arrival counters in
+ * the workspace.  It sums w13
  * over the whole K range in one fp32 chain, so its result equals the
  * multi-launch path's (MOE_DISABLE_FUSED=1 in the environment selects that
  * path) bit for bit where that path leaves w13 unsplit (H < 512), and up to
@@ -140,8 +142,8 @@ moe_status_t moe_forward(const moe_bf16_t* x, const float* logits, const moe_bf1
  * events[i] (cudaEvent_t, created by the caller) on `stream` at the stage
  * boundaries: [0] before routing, [1] after route+permute, [2] after the
  * w13/SwiGLU kernel, [3] after the w2 kernel, [4] after the combine.  n_events
- * must be 5.  When the FFN and combine are one launch (moe_forward_fused),
- * events [2], [3] and [4] are all recorded after it.  A recorded event is a
+ * must be 5.  When the layer is one launch (moe_forward_fused), [1] is
+ * recorded right after [0] and [2], [3] and [4] after the launch.  A recorded event is a
  * stream operation, so the launch overlap between the stages it separates is
  * lost while measuring. */
 moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const moe_bf16_t* w13,
@@ -188,7 +190,7 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
  * bf16 exactly on chip (into tensor memory, the MMA's A operand), so the
  * tensor-core products are those of the bf16 path; each weight row's scale
  * multiplies its fp32 accumulator row.  Runs
- * only as the one-launch FFN (moe_forward_w8_supported; 2 kernels):
+ * only as the one-launch layer (moe_forward_w8_supported; 1 kernel):
  * MOE_ERR_UNSUPPORTED_SHAPE otherwise, whatever MOE_DISABLE_FUSED says.  Codes
  * 0x7F / 0xFF (NaN) propagate as NaN.  All pointers 16-byte aligned. */
 moe_status_t moe_forward_w8(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
@@ -197,8 +199,8 @@ moe_status_t moe_forward_w8(const moe_bf16_t* x, const float* logits, const uint
                             float* topk_weights, int32_t* expert_offsets, int32_t* permuted_rows,
                             void* workspace, size_t ws_bytes, moe_stream_t stream);
 
-/* moe_forward_w8 recording the 5 stage events of moe_forward_timed ([2] .. [4]
- * all mark the end of the one FFN + combine launch). */
+/* moe_forward_w8 recording the 5 stage events of moe_forward_timed ([0] and [1]
+ * before its one launch, [2] .. [4] after it). */
 moe_status_t moe_forward_w8_timed(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
                                   const float* w13_scale, const uint8_t* w2,
                                   const float* w2_scale, moe_shape_t shape, moe_bf16_t* out,
@@ -207,7 +209,7 @@ moe_status_t moe_forward_w8_timed(const moe_bf16_t* x, const float* logits, cons
                                   void* workspace, size_t ws_bytes, moe_stream_t stream,
                                   void* const* events, int n_events);
 
-/* 1 if moe_forward_w8 accepts `shape` (the one-launch FFN's shapes), else 0. */
+/* 1 if moe_forward_w8 accepts `shape` (the one-launch layer's shapes), else 0. */
 int moe_forward_w8_supported(moe_shape_t shape);
 
 /* Number of kernels one moe_forward call launches for `shape` (0 if unsupported). */
@@ -225,8 +227,8 @@ int moe_forward_kernel_count(moe_shape_t shape);
 moe_status_t moe_selftest_wait_timeout(void* workspace, size_t ws_bytes, unsigned limit_us,
                                        moe_stream_t stream);
 
-/* 1 if moe_forward runs w13, w2 and the combine of `shape` as one persistent
- * launch (T <= 64 and T*k <= 4096, unless MOE_DISABLE_FUSED=1), else 0. */
+/* 1 if moe_forward runs the whole layer of `shape` as one persistent launch
+ * (T <= 64, unless MOE_DISABLE_FUSED=1), else 0. */
 int moe_forward_fused(moe_shape_t shape);
 
 /* Waits for `stream`, then reads and clears the device error word kept in the
