@@ -75,6 +75,21 @@ using namespace gemm;
 constexpr int kMaxK = 16;       // combine: selected experts per token
 constexpr int kMaxSplits = 8;   // split-K slices per GEMM
 
+// The routing every CTA does for itself (one-launch FFN: at most 64 tokens, so at
+// most 1024 expanded rows, and at most 1024 experts): permuted rows, routing
+// weights by expanded row, expert offsets, and the expert of each tile (every
+// expert's rows fit one tile, so tile j is the j-th touched expert).  After the
+// unit table in shared memory.
+constexpr int kMaxRows = kMaxK * 64;
+constexpr int kMaxExperts = 1024;
+struct alignas(16) RouteSmem {
+    int16_t rows[kMaxRows];
+    int16_t tile_expert[kMaxExperts];
+    int16_t off[kMaxExperts + 8];
+    float w[kMaxRows];
+    int n_tiles;
+};
+
 struct FusedArgs {
     const __nv_bfloat16* x;       // [T, H]
     const float* logits;          // [T, E]
@@ -127,20 +142,6 @@ struct ComboScratch {
     float w[kMaxK];
 };
 
-// The routing every CTA does for itself (one-launch FFN: at most 64 tokens, so at
-// most 1024 expanded rows, and at most 1024 experts): permuted rows, routing
-// weights by expanded row, expert offsets, and the expert of each tile (every
-// expert's rows fit one tile, so tile j is the j-th touched expert).  After the
-// unit table in shared memory.
-constexpr int kMaxRows = kMaxK * 64;
-constexpr int kMaxExperts = 1024;
-struct alignas(16) RouteSmem {
-    int16_t rows[kMaxRows];
-    int16_t tile_expert[kMaxExperts];
-    int16_t off[kMaxExperts + 8];
-    float w[kMaxRows];
-    int n_tiles;
-};
 constexpr int kFusedReserve = kUnitTableBytes + (int)sizeof(RouteSmem);
 
 template <int NT>
@@ -264,124 +265,182 @@ __device__ __forceinline__ bool wait_counters(const FusedArgs& a, volatile int* 
 
 // Routes the T tokens in this CTA (every thread calls; ends with a barrier).
 // scratch: shared memory unused until the producer starts, at least
-// route_scratch_bytes(warps) bytes.  Per token one warp stages its E logits in
-// shared memory, then takes the k experts in k rounds of warp arg-max over the
-// experts not yet taken (larger logit first, then the lower expert: the order of
-// the routing kernels), lane j keeping the j-th; the weights are those kernels'
-// softmax, bit for bit.  Then per-expert counts, offsets (a block scan), the
-// tiles (touched experts in order) and the stable permutation (one warp, rows in
-// ascending order, ranks from peer masks).  CTA 0 also writes the user-visible
+// kRouteScratchBytes.  The logits are staged in shared memory -- all T rows with
+// one cooperative load when they fit in kStagedLogitBytes, else one row per warp
+// at a time -- and each token is selected by one warp in two passes, as in the
+// routing kernels: tau = the k-th largest of the 32 lanes' maxima; the experts
+// whose logit reaches tau (usually about a dozen) are sorted by (logit desc,
+// expert asc) and the first k kept, lane j holding the j-th (more than 32 such
+// experts, from ties, or a small k over few experts: k rounds of warp arg-max
+// instead).  The weights are those
+// kernels' softmax, bit for bit.  Each selection sets bit t of its expert's
+// 64-bit token mask (T <= 64).  Then one block scan gives the expert offsets and
+// the tiles (touched experts in order), and every expanded row r = t k + j of
+// expert e goes to offsets[e] + popc(mask[e] & (2^t - 1)): the stable order
+// (ascending r within an expert, because an expert appears at most once per
+// token), each row placed independently.  CTA 0 also writes the user-visible
 // routing outputs.
-constexpr int route_scratch_bytes(int warps)
+constexpr int kStagedLogitBytes = 128 * 1024;
+constexpr int kRouteScratchBytes =
+    kStagedLogitBytes + kMaxExperts * 8 + (kMaxRows + 32) * 4 + 20 * 32 * 8;
+
+// The two-pass selection; false (nothing selected) when more than 32 experts
+// reach tau.
+__device__ __forceinline__ bool select_by_threshold(const float* row, int E, int k, int lane,
+                                                    float2* cand, float& my_l, int& my_e)
 {
-    return warps * kMaxExperts * 4 + (kMaxExperts + kMaxRows + 32) * 4;
+    const int M = (E + 31) / 32;  // slot m of lane l: expert 32 m + l
+    float mv = -INFINITY;
+    for (int m = 0; m < M; ++m) {
+        const int e = m * 32 + lane;
+        if (e < E) mv = fmaxf(mv, row[e]);
+    }
+    const float tau = warp_kth_largest(mv, k);
+    uint32_t mask = 0;
+    for (int m = 0; m < M; ++m) {
+        const int e = m * 32 + lane;
+        if (e < E && row[e] >= tau) mask |= 1u << m;
+    }
+    const int c = __popc(mask);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += n;
+    }
+    const int total = __shfl_sync(kFull, incl, 31);
+    if (total > 32) return false;
+    int pos = incl - c;
+    while (mask) {
+        const int m = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int e = m * 32 + lane;
+        cand[pos++] = make_float2(row[e], __int_as_float(e));
+    }
+    __syncwarp();
+    sort_candidates(total, lane, cand, my_l, my_e);
+    return true;
+}
+
+__device__ __forceinline__ void select_token(const float* row, int E, int k, int lane,
+                                             float2* cand, float& my_l, int& my_e)
+{
+    const int M = (E + 31) / 32;  // slot m of lane l: expert 32 m + l
+    // few rounds over few slots (tiny layers): the k rounds of arg-max below are
+    // the shorter dependency chain
+    const bool rounds = k * (M + 10) <= 2 * M + 25;
+    if (!rounds && select_by_threshold(row, E, k, lane, cand, my_l, my_e)) return;
+    // k rounds of warp arg-max over the experts not yet taken (also the exact
+    // fallback when more than 32 experts reach tau)
+    uint32_t taken = 0;  // bit m: expert 32 m + lane already selected
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int be = kNoIndex;
+        for (int m = 0; m < M; ++m) {  // experts ascend, so '>' keeps the lower one
+            const int e = m * 32 + lane;
+            if (e < E && !((taken >> m) & 1u)) {
+                const float v = row[e];
+                if (be == kNoIndex || v > bv) {
+                    bv = v;
+                    be = e;
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(kFull, bv, off);
+            const int oi = __shfl_xor_sync(kFull, be, off);
+            if (key_before(ov, oi, bv, be)) {
+                bv = ov;
+                be = oi;
+            }
+        }
+        if (lane == j) {
+            my_l = bv;
+            my_e = be;
+        }
+        if (be != kNoIndex && (be & 31) == lane) taken |= 1u << (be >> 5);
+    }
 }
 
 __device__ __forceinline__ void route_tokens(const FusedArgs& a, RouteSmem* rs, uint8_t* scratch)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    float* myrow = reinterpret_cast<float*>(scratch) + warp * kMaxExperts;
-    int* cnt = reinterpret_cast<int*>(scratch) + nwarps * kMaxExperts;  // [E], later cursors
-    int* ids_s = cnt + kMaxExperts;                                     // [R]
-    int* sums = ids_s + kMaxRows;                                       // [32]
+    float* logits_s = reinterpret_cast<float*>(scratch);
+    unsigned long long* tmask =
+        reinterpret_cast<unsigned long long*>(scratch + kStagedLogitBytes);  // [E]
+    int* ids_s = reinterpret_cast<int*>(tmask + kMaxExperts);               // [R]
+    int* sums = ids_s + kMaxRows;                                           // [32]
+    float2* cand = reinterpret_cast<float2*>(sums + 32) + warp * 32;        // [warps][32]
     const int E = a.E, k = a.k;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    const bool all_rows = (long)a.T * E * 4 <= kStagedLogitBytes;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) tmask[e] = 0ull;
+    if (all_rows) {
+        const long n = (long)a.T * E;
+        if ((E & 3) == 0) {
+            for (long i = threadIdx.x; i < n / 4; i += blockDim.x)
+                reinterpret_cast<float4*>(logits_s)[i] =
+                    __ldg(reinterpret_cast<const float4*>(a.logits) + i);
+        } else {
+            for (long i = threadIdx.x; i < n; i += blockDim.x) logits_s[i] = __ldg(a.logits + i);
+        }
+    }
     __syncthreads();
-    const int M = (E + 31) / 32;
     for (int t = warp; t < a.T; t += nwarps) {
-        const float* src = a.logits + (size_t)t * E;
-        for (int e = lane; e < E; e += 32) myrow[e] = __ldg(src + e);
-        __syncwarp();
-        uint32_t taken = 0;  // bit m: expert 32 m + lane already selected
+        const float* row = logits_s + (size_t)t * E;
+        if (!all_rows) {  // this warp's row buffer (E <= 1024 floats each)
+            float* myrow = logits_s + (size_t)warp * kMaxExperts;
+            const float* src = a.logits + (size_t)t * E;
+            for (int e = lane; e < E; e += 32) myrow[e] = __ldg(src + e);
+            __syncwarp();
+            row = myrow;
+        }
         float my_l = -INFINITY;
         int my_e = 0;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int be = kNoIndex;
-            for (int m = 0; m < M; ++m) {  // experts ascend, so '>' keeps the lower one
-                const int e = m * 32 + lane;
-                if (e < E && !((taken >> m) & 1u)) {
-                    const float v = myrow[e];
-                    if (be == kNoIndex || v > bv) {
-                        bv = v;
-                        be = e;
-                    }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(kFull, bv, off);
-                const int oi = __shfl_xor_sync(kFull, be, off);
-                if (key_before(ov, oi, bv, be)) {
-                    bv = ov;
-                    be = oi;
-                }
-            }
-            if (lane == j) {
-                my_l = bv;
-                my_e = be;
-            }
-            if (be != kNoIndex && (be & 31) == lane) taken |= 1u << (be >> 5);
-        }
-        const float w = softmax_weight(my_l, k, lane);
+        select_token(row, E, k, lane, cand, my_l, my_e);
+    const float w = softmax_weight(my_l, k, lane);
         if (lane < k) {
             const int r = t * k + lane;
             ids_s[r] = my_e;
             rs->w[r] = w;
-            atomicAdd(&cnt[my_e], 1);
+            atomicOr(&tmask[my_e], 1ull << t);
             if (blockIdx.x == 0) {
                 a.ids_out[r] = my_e;
                 a.weights_out[r] = w;
             }
         }
-        __syncwarp();  // myrow is rewritten for the warp's next token
+        __syncwarp();  // the row buffer and cand are rewritten for the warp's next token
     }
     __syncthreads();
-    // offsets and tiles: thread i owns experts 2 i and 2 i + 1 (blockDim >= E / 2)
+    // offsets and tiles in one scan: thread i owns experts 2 i and 2 i + 1
+    // (blockDim >= E / 2); the low 16 bits count rows, the high ones tiles
     const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
-    const int c0 = e0 < E ? cnt[e0] : 0, c1 = e1 < E ? cnt[e1] : 0;
-    int total, ntiles;
-    const int base = block_exclusive_scan(c0 + c1, sums, total);
-    const int tbase = block_exclusive_scan((c0 > 0) + (c1 > 0), sums, ntiles);
+    const int c0 = e0 < E ? __popcll(tmask[e0]) : 0, c1 = e1 < E ? __popcll(tmask[e1]) : 0;
+    int packed_total;
+    const int packed = block_exclusive_scan((c0 + c1) | (((c0 > 0) + (c1 > 0)) << 16), sums,
+                                            packed_total);
+    const int base = packed & 0xffff, tbase = packed >> 16;
     if (e0 < E) {
         rs->off[e0] = (int16_t)base;
-        cnt[e0] = base;  // the cursor of the stable scatter
         if (c0) rs->tile_expert[tbase] = (int16_t)e0;
         if (blockIdx.x == 0) a.offsets_out[e0] = base;
     }
     if (e1 < E) {
         rs->off[e1] = (int16_t)(base + c0);
-        cnt[e1] = base + c0;
         if (c1) rs->tile_expert[tbase + (c0 > 0)] = (int16_t)e1;
         if (blockIdx.x == 0) a.offsets_out[e1] = base + c0;
     }
     if (threadIdx.x == 0) {
-        rs->off[E] = (int16_t)total;
-        rs->n_tiles = ntiles;
-        if (blockIdx.x == 0) a.offsets_out[E] = total;
+        rs->off[E] = (int16_t)(packed_total & 0xffff);
+        rs->n_tiles = packed_total >> 16;
+        if (blockIdx.x == 0) a.offsets_out[E] = packed_total & 0xffff;
     }
     __syncthreads();
-    if (warp == 0) {
-        const unsigned lt = (1u << lane) - 1u;
-        for (int r0 = 0; r0 < a.R; r0 += 32) {
-            const int r = r0 + lane;
-            const bool valid = r < a.R;
-            const int e = valid ? ids_s[r] : -1;
-            const unsigned vm = __ballot_sync(kFull, valid);
-            unsigned peers = 0;
-            int pos = 0;
-            if (valid) {
-                peers = __match_any_sync(vm, e);
-                pos = cnt[e] + __popc(peers & lt);
-            }
-            __syncwarp();
-            if (valid) {
-                rs->rows[pos] = (int16_t)r;
-                if (blockIdx.x == 0) a.rows_out[pos] = r;
-                if (lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
-            }
-            __syncwarp();
-        }
+    for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+        const int e = ids_s[r], t = r / k;
+        const int pos = rs->off[e] + __popcll(tmask[e] & ((1ull << t) - 1ull));
+        rs->rows[pos] = (int16_t)r;
+        if (blockIdx.x == 0) a.rows_out[pos] = r;
     }
     __syncthreads();
 }
@@ -411,7 +470,9 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     int4* unit_tab = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(aux) + C::kAuxBytes);
     int* tab_seq = reinterpret_cast<int*>(unit_tab + 2 * kUnitTable);
     RouteSmem* rs = reinterpret_cast<RouteSmem*>(tab_seq + kUnitTable);
-    static_assert(route_scratch_bytes((W8 ? R8::kThreads : kThreads) / 32) <= kRingBytes,
+    static_assert(kRouteScratchBytes <= kRingBytes &&
+                      (W8 ? R8::kThreads : kThreads) / 32 * kMaxExperts * 4 <= kStagedLogitBytes &&
+                      (W8 ? R8::kThreads : kThreads) / 32 <= 20,
                   "routing scratch");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1275,13 +1336,14 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     a.min_kt_per_split = 4;
     a.s13 = b.s13;
     a.s2 = b.s2;
+    const int grid = plan.grid;
     switch (plan.nt * 2 + (w8 ? 1 : 0)) {
-    case 32: return launch_fused_nt<16, false>(t13, t2, ta, a, plan.grid, st);
-    case 64: return launch_fused_nt<32, false>(t13, t2, ta, a, plan.grid, st);
-    case 128: return launch_fused_nt<64, false>(t13, t2, ta, a, plan.grid, st);
-    case 33: return launch_fused_nt<16, true>(t13, t2, ta, a, plan.grid, st);
-    case 65: return launch_fused_nt<32, true>(t13, t2, ta, a, plan.grid, st);
-    case 129: return launch_fused_nt<64, true>(t13, t2, ta, a, plan.grid, st);
+    case 32: return launch_fused_nt<16, false>(t13, t2, ta, a, grid, st);
+    case 64: return launch_fused_nt<32, false>(t13, t2, ta, a, grid, st);
+    case 128: return launch_fused_nt<64, false>(t13, t2, ta, a, grid, st);
+    case 33: return launch_fused_nt<16, true>(t13, t2, ta, a, grid, st);
+    case 65: return launch_fused_nt<32, true>(t13, t2, ta, a, grid, st);
+    case 129: return launch_fused_nt<64, true>(t13, t2, ta, a, grid, st);
     default: return cudaErrorInvalidValue;
     }
 }

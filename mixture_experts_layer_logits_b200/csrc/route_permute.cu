@@ -29,29 +29,6 @@ namespace moe {
 namespace {
 
 
-// Sorts one (value, index) key per lane across groups of W lanes (W = 16: each
-// half-warp on its own; W = 32: the warp) so that the group's first lane holds
-// the key that ranks first (larger value, then lower index).  Bitonic network with
-// the "ranks before" relation as the order; keys must be distinct (they are:
-// indices are unique).
-template <int W>
-__device__ __forceinline__ void warp_sort_keys(float& v, int& i, int lane)
-{
-#pragma unroll
-    for (int size = 2; size <= W; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const float ov = __shfl_xor_sync(kFull, v, stride);
-            const int oi = __shfl_xor_sync(kFull, i, stride);
-            const bool take_first = ((lane & stride) == 0) == ((lane & size) == 0);
-            if (take_first == key_before(ov, oi, v, i)) {
-                v = ov;
-                i = oi;
-            }
-        }
-    }
-}
-
 // Sorts one float per lane across the warp, largest in lane 0.
 __device__ __forceinline__ float warp_sort_desc(float v, int lane)
 {
@@ -109,55 +86,6 @@ __device__ __forceinline__ void warp_load_row(const float* __restrict__ row, int
             v[m] = (e < E) ? __ldg(row + e) : -INFINITY;
         }
     }
-}
-
-// Float -> unsigned key with the same order (-0.0 and +0.0 map to one key), and
-// back.  Key 0 stands below every non-NaN value.
-__device__ __forceinline__ uint32_t ordered_key(float f)
-{
-    const uint32_t b = __float_as_uint(f + 0.0f);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float key_value(uint32_t key)
-{
-    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
-}
-
-// The k-th largest (k >= 1, duplicates counted) of the warp's 32 values: at most
-// k rounds of a warp max reduction, each removing the lanes that hold the max.
-__device__ __forceinline__ float warp_kth_largest(float x, int k)
-{
-    uint32_t key = ordered_key(x);
-    int left = k;
-    for (;;) {
-        const uint32_t m = __reduce_max_sync(kFull, key);
-        left -= __popc(__ballot_sync(kFull, key == m));
-        if (left <= 0) return key_value(m);
-        if (key == m) key = 0;
-    }
-}
-
-// Sorts the candidates cand[0 .. total) (total <= 32, distinct experts) by (logit
-// desc, expert asc) and leaves the j-th in lane j: (my_l, my_id).
-__device__ __forceinline__ void sort_candidates(int total, int lane, const float2* cand,
-                                                float& my_l, int& my_id)
-{
-    float cv = -INFINITY;
-    int ci = kNoIndex - lane;  // distinct sentinels rank after every expert
-    if (lane < total) {
-        const float2 cc = cand[lane];
-        cv = cc.x;
-        ci = __float_as_int(cc.y);
-    }
-    __syncwarp();  // cand may be rewritten by this warp's next token
-    // usually about k candidates: then lanes 0..15 hold all of them and a
-    // half-warp network (10 stages instead of 15) orders them the same way
-    if (total <= 16)
-        warp_sort_keys<16>(cv, ci, lane);
-    else
-        warp_sort_keys<32>(cv, ci, lane);
-    my_l = cv;
-    my_id = ci;
 }
 
 // Exact selection when more than 32 experts reach the threshold (ties, -inf
