@@ -54,8 +54,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (workload, kernel).  An entry is removed when its kernel changes, until it is
 # captured again.
 NCU_TRAFFIC = {
-    ("decode", "fused_ffn"): 509_740_032 + 4_323_328,
-    ("decode+e4m3", "fused_ffn"): 257_047_040 + 3_710_976,
+    ("prefill", "w13"): 3_694_407_168 + 205_702_912,
+    ("prefill", "w2"): 1_829_378_048 + 509_899_264,
+    ("decode", "fused_ffn"): 509_752_832 + 3_875_328,
+    ("decode+e4m3", "fused_ffn"): 257_118_464 + 3_917_056,
+    ("routing_stress", "route"): 67_143_424 + 793_344,
 }
 
 # Records added to the default line (workload name, expert weight format).
