@@ -465,7 +465,7 @@ def routing_bench(args, w, ctx, K, W, cpu_seconds):
     peaks, peak_kind = load_peaks()
     route_bytes = T * E * 4 + R * 8
     perm_bytes = R * 4 + (E + 1) * 4 + R * 4
-    launches = 1 + (1 if R <= 4096 else 3)  # route; one permute kernel, or count + scan + scatter
+    launches = 2  # the route kernel, then one permutation kernel (one CTA, or the whole grid)
     ck = clocks.report()
     # The routing kernel reads the logits, the dominant traffic of the step; the
     # permutation kernels move about 1 MB and are latency-bound.

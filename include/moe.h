@@ -91,7 +91,15 @@ moe_status_t moe_route(const float* logits, moe_shape_t shape, int32_t* topk_ids
                        float* topk_weights, moe_stream_t stream);
 
 /* permute.  topk_ids int32 [T*k] (values in [0, E)) -> expert_offsets int32 [E+1],
- * permuted_rows int32 [T*k].  Ids outside [0, E) are outside the contract. */
+ * permuted_rows int32 [T*k].  Ids outside [0, E) are outside the contract.
+ * Up to 4096 rows one CTA does the whole permutation.  Beyond that it is one
+ * launch of at most one CTA per SM whose CTAs meet at two grid barriers (the
+ * chunk counts must all be in before the prefixes over the chunks are formed,
+ * and those before any row is placed); the workspace holds the count table and
+ * the barrier.  Co-residency: as for the one-launch layer (moe_forward), the
+ * launch assumes all of its CTAs run at once; every wait is bounded (2 s, then
+ * moe_device_status reports MOE_ERR_DEVICE_TIMEOUT and the outputs are
+ * unspecified), so it never hangs. */
 moe_status_t moe_permute(const int32_t* topk_ids, moe_shape_t shape, int32_t* expert_offsets,
                          int32_t* permuted_rows, void* workspace, size_t ws_bytes,
                          moe_stream_t stream);
@@ -160,7 +168,7 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
  * computes (same kernels, same bit-exact result).
  *
  * Scratch: a file-scope device array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES
- * (about 2 MiB) inside the library; every GPU on which the library is used holds
+ * (about 1 MiB) inside the library; every GPU on which the library is used holds
  * it until the process exits.  The caller still passes topk_ids, expert_offsets
  * and permuted_rows (device pointers, 16-byte aligned).
  * Limits: T*k <= MOE_PERMUTE_NOALLOC_MAX_ROWS and the moe_permute shape rules,
@@ -175,7 +183,7 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* logits, const m
  * threads, same device) race and may return wrong results; order them on one
  * stream. */
 #define MOE_PERMUTE_NOALLOC_MAX_ROWS (1 << 20)
-#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (2097152 + 4096 + 32768 + 256)
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (1052672 + 32768 + 256)
 moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
                                  int32_t* expert_offsets, int32_t* permuted_rows,
                                  moe_stream_t stream);

@@ -235,18 +235,6 @@ __device__ __forceinline__ bool warp_wait_count(const int32_t* ctr, int target,
     }
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p)
-{
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v)
-{
-    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
 // Bounded wait until CTA 0 has zeroed this call's arrival counters (*ready ==
 // gen, read with acquire).  False on a timeout, a local abort or another CTA's
 // recorded error.

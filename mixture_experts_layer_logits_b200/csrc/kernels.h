@@ -51,15 +51,40 @@ struct Tile {
     int pad[3];
 };
 
+// The grid barrier of the multi-CTA permutation (32 bytes of device memory;
+// needs no initialisation).  CTA 0 of a call zeroes `count`, then publishes the
+// call's generation in `gen` (release); every CTA waits for that before its
+// first arrival.  A CTA that gives up on a wait stores the call's generation in
+// `abort`, so the others stop too.
+struct GridBar {
+    uint32_t count;
+    uint32_t pad;
+    unsigned long long gen;
+    unsigned long long abort;
+    unsigned long long pad2;
+};
+
 // Everything the route/permute kernels write besides the user-visible outputs.
 struct PermuteAux {
     Tile* tiles;           // [max_tiles]
     int32_t* num_tiles;    // device scalar
     int nt;                // token rows per tile (the GEMM's N tile)
-    int32_t* chunk_counts; // [n_chunks + 1, E] scratch of the multi-CTA path
-    int32_t* err;          // the error word (debug-build index checks); may be null
+    int32_t* err;          // the error word (bounded-wait timeouts, debug-build index checks)
     int max_tiles;         // entries of `tiles`
+    int32_t* chunk_counts; // [max_chunks + 1, E] scratch of the multi-CTA path
+    int max_chunks;        // its chunk rows (the multi-CTA path's grid bound)
+    GridBar* bar;          // the multi-CTA path's grid barrier
+    unsigned long long gen;  // a value unique to this call (next_generation())
 };
+
+// A value unique to each call that synchronises CTAs through workspace words
+// (the one-launch FFN, the multi-CTA permutation): a per-process random start
+// plus a counter, so that neither an earlier call's value nor stale workspace
+// bytes match it.
+unsigned long long next_generation();
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sms();
 
 // Records the cudaError_t that moe_last_cuda_error() reports on this host thread.
 void set_last_cuda_error(int err);
@@ -102,13 +127,14 @@ cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k,
                                        float* weights, int32_t* offsets, int32_t* rows,
                                        const PermuteAux& aux, cudaStream_t st);
 
-// Multi-CTA path: per-chunk counts, per-expert prefixes over the chunks (and the
-// expert totals), then a per-chunk stable scatter (CTA 0 also writes offsets and
-// tiles).
-constexpr int kChunkRows = 2048;
+// Multi-CTA path, one launch of at most min(SMs, aux.max_chunks) CTAs that must
+// all be resident at once: every CTA counts and ranks its chunk of rows, then
+// (after a grid barrier) the per-expert prefixes over the chunks are formed, and
+// (after a second) every CTA places its chunk stably; the CTAs also write the
+// offsets and the tile list.  Waits are bounded (2 s, then kDeviceErrorMagic in
+// aux.err).
 cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                                  int32_t* rows, const PermuteAux& aux, cudaStream_t st);
-size_t large_permute_smem(int E);
 
 // Tile list from expert_offsets alone (moe_grouped_ffn called on its own).
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int R, const PermuteAux& aux,

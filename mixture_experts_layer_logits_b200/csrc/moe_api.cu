@@ -79,8 +79,9 @@ bool combine_shape_ok(const moe_shape_t& s)
 }
 
 struct Layout {
-    size_t err, ids, weights, offsets, rows, tiles, num_tiles, splits, chunks, partials, act, y,
-        partials2, counters, ready, total;
+    size_t err, ids, weights, offsets, rows, tiles, num_tiles, splits, chunks, bar, partials, act,
+        y, partials2, counters, ready, total;
+    int max_chunks;  // chunk rows of the multi-CTA permutation's count table
     FfnPlan plan;
     bool ffn;
     bool fused;      // the shape qualifies for the one-launch FFN + combine
@@ -108,9 +109,11 @@ Layout layout_for(const moe_shape_t& s)
     L.tiles = take((size_t)L.plan.max_tiles * sizeof(Tile));
     L.num_tiles = take(sizeof(int32_t));
     L.splits = take(2 * sizeof(int32_t));
-    // per-chunk expert counts (then prefixes), plus one row of expert totals
-    const size_t n_chunks = (R + kChunkRows - 1) / kChunkRows;
-    L.chunks = take((n_chunks + 1) * (size_t)s.E * sizeof(int32_t));
+    // multi-CTA permutation: per-chunk expert counts (then prefixes over the
+    // chunks), one row of expert totals, and its grid barrier
+    L.max_chunks = R > (size_t)kSmallRows ? kSizingSms : 0;
+    L.chunks = take((size_t)(L.max_chunks + 1) * s.E * sizeof(int32_t));
+    L.bar = take(sizeof(GridBar));
     if (L.ffn) {
         size_t p13 = L.plan.s13_max > 1 ? (size_t)L.plan.s13_max * R * 2 * I : 0;
         size_t p2 = L.plan.s2_max > 1 ? (size_t)L.plan.s2_max * R * H : 0;
@@ -137,6 +140,8 @@ T* at(void* ws, size_t off)
     return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
 
+}  // namespace
+
 int device_sms()
 {
     static int cached[64] = {0};
@@ -151,6 +156,8 @@ int device_sms()
     return cached[dev];
 }
 
+namespace {
+
 moe_status_t cuda_status(cudaError_t e)
 {
     if (e == cudaSuccess) return MOE_OK;
@@ -158,15 +165,32 @@ moe_status_t cuda_status(cudaError_t e)
     return MOE_ERR_CUDA;
 }
 
+}  // namespace
+
+unsigned long long next_generation()
+{
+    static std::atomic<unsigned long long> counter{[] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 32) ^ rd() ^
+               (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    }()};
+    return counter.fetch_add(0x9E3779B97F4A7C15ull) + 0x9E3779B97F4A7C15ull;
+}
+
+namespace {
+
 PermuteAux make_aux(void* ws, const Layout& L, const moe_shape_t& s)
 {
     PermuteAux a;
     a.tiles = at<Tile>(ws, L.tiles);
     a.num_tiles = at<int32_t>(ws, L.num_tiles);
     a.nt = L.plan.nt;
-    a.chunk_counts = at<int32_t>(ws, L.chunks);
     a.err = at<int32_t>(ws, L.err);
     a.max_tiles = L.plan.max_tiles;
+    a.chunk_counts = at<int32_t>(ws, L.chunks);
+    a.max_chunks = L.max_chunks;
+    a.bar = at<GridBar>(ws, L.bar);
+    a.gen = next_generation();
     (void)s;
     return a;
 }
@@ -187,20 +211,6 @@ moe_status_t run_permute(const float* logits, int32_t* ids, float* weights, cons
         if (e == cudaSuccess) e = launch_large_permute(ids, s.T, s.E, s.top_k, offsets, rows, aux, st);
     }
     return cuda_status(e);
-}
-
-// A value unique to each one-launch FFN call (the generation its CTA 0 publishes
-// once the call's counters are zeroed): a per-process random start plus a
-// counter, so that neither an earlier call's value nor stale workspace bytes
-// match it.
-unsigned long long next_generation()
-{
-    static std::atomic<unsigned long long> counter{[] {
-        std::random_device rd;
-        return ((unsigned long long)rd() << 32) ^ rd() ^
-               (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
-    }()};
-    return counter.fetch_add(0x9E3779B97F4A7C15ull) + 0x9E3779B97F4A7C15ull;
 }
 
 moe_status_t run_ffn(const void* x, const void* w13, const void* w2, const int32_t* rows,
@@ -440,8 +450,9 @@ int moe_forward_kernel_count(moe_shape_t s)
     const Layout L = layout_for(s);
     // the one-launch FFN routes and permutes inside its own launch
     if (L.fused && fused_enabled()) return 1;
-    // routing and permutation: one kernel, or route + count + prefix + scatter
-    const int route_permute = R <= kSmallRows ? 1 : 4;
+    // routing and permutation: one kernel, or the route kernel + the one-launch
+    // multi-CTA permutation
+    const int route_permute = R <= kSmallRows ? 1 : 2;
     // w13, [SwiGLU finalize], w2, combine
     return route_permute + 2 + (L.plan.s13_max > 1 ? 1 : 0) + 1;
 }

@@ -2,9 +2,9 @@
 // without a caller-supplied workspace, for callers that cannot allocate device
 // memory.
 //
-// The scratch the permutation kernels need (the per-chunk expert count table of
-// the multi-CTA path, and the per-expert tile list they also emit) lives in one
-// file-scope device array of fixed size.  Host code cannot use the array's name
+// The scratch the permutation kernels need (the per-chunk expert count table and
+// the grid barrier of the multi-CTA path, and the per-expert tile list they also
+// emit) lives in one file-scope device array of fixed size.  Host code cannot use the array's name
 // as a device address, so its address is looked up with cudaGetSymbolAddress
 // once per device, with that device current, and handed to the kernels like any
 // other pointer.  Nothing here allocates.
@@ -19,13 +19,15 @@
 namespace moe {
 namespace {
 
-// chunk count table for MOE_PERMUTE_NOALLOC_MAX_ROWS / kChunkRows chunks x 1024 experts
-// plus its row of expert totals, then up to 1024 tiles (one per expert), then the
-// tile count
-constexpr size_t kMaxChunks = (MOE_PERMUTE_NOALLOC_MAX_ROWS + kChunkRows - 1) / kChunkRows;
-constexpr size_t kCountBytes = (kMaxChunks + 1) * 1024 * sizeof(int32_t);
+// chunk count table for up to 256 chunks (the multi-CTA path's grid bound) x 1024
+// experts plus its row of expert totals, then up to 1024 tiles (one per expert),
+// then a 256-byte tail: the tile count at +0, the error word at +16, the grid
+// barrier at +64
+constexpr int kMaxChunks = 256;
+constexpr size_t kCountBytes = (size_t)(kMaxChunks + 1) * 1024 * sizeof(int32_t);
 constexpr size_t kTileBytes = 1024 * sizeof(Tile);
 constexpr size_t kScratchBytes = kCountBytes + kTileBytes + 256;
+static_assert(64 + sizeof(GridBar) <= 256, "tail layout");
 static_assert(kScratchBytes == MOE_PERMUTE_NOALLOC_SCRATCH_BYTES, "header and file disagree");
 
 static __device__ __align__(256) unsigned char g_permute_scratch[kScratchBytes];
@@ -76,10 +78,14 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t
         aux.chunk_counts = reinterpret_cast<int32_t*>(p);
         aux.tiles = reinterpret_cast<Tile*>(p + kCountBytes);
         aux.num_tiles = reinterpret_cast<int32_t*>(p + kCountBytes + kTileBytes);
-        // debug build: index faults are recorded here (nothing reports them)
+        // bounded-wait timeouts and debug-build index faults are recorded here
+        // (nothing reports them)
         aux.err = reinterpret_cast<int32_t*>(p + kCountBytes + kTileBytes + 16);
         aux.nt = 1 << 30;  // one tile per expert: the tile list stays within 1024 entries
         aux.max_tiles = 1024;
+        aux.max_chunks = kMaxChunks;
+        aux.bar = reinterpret_cast<GridBar*>(p + kCountBytes + kTileBytes + 64);
+        aux.gen = next_generation();
         cudaStream_t st = static_cast<cudaStream_t>(stream);
         int32_t* ids = const_cast<int32_t*>(topk_ids);
         if (R <= kSmallRows)

@@ -52,6 +52,19 @@ __device__ __forceinline__ void red_release_gpu_add(int* p, int v)
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// 64-bit acquire load / release store at GPU scope (generation flags).
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 // Orders this thread's generic-proxy global accesses with its async-proxy ones
 // (TMA) on either side of the fence.
 __device__ __forceinline__ void fence_proxy_async_global()

@@ -150,4 +150,41 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sums, int& total
     return prefix + incl - v;
 }
 
+// block_exclusive_scan of a pair of ints (both members scanned at once).
+// `sums` is shared scratch of 32 int2.
+__device__ __forceinline__ int2 block_exclusive_scan2(int2 v, int2* sums, int2& total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int2 incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int nx = __shfl_up_sync(kFull, incl.x, off);
+        const int ny = __shfl_up_sync(kFull, incl.y, off);
+        if (lane >= off) {
+            incl.x += nx;
+            incl.y += ny;
+        }
+    }
+    if (lane == 31) sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int2 s = (lane < nw) ? sums[lane] : make_int2(0, 0);
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int nx = __shfl_up_sync(kFull, s.x, off);
+            const int ny = __shfl_up_sync(kFull, s.y, off);
+            if (lane >= off) {
+                s.x += nx;
+                s.y += ny;
+            }
+        }
+        sums[lane] = s;
+    }
+    __syncthreads();
+    const int2 prefix = (warp > 0) ? sums[warp - 1] : make_int2(0, 0);
+    total = sums[nw - 1];
+    __syncthreads();
+    return make_int2(prefix.x + incl.x - v.x, prefix.y + incl.y - v.y);
+}
+
 }  // namespace moe

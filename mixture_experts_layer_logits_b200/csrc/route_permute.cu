@@ -11,10 +11,12 @@
 // per-lane value count V (a template), and the grid scales with T.
 //
 // Permutation: count -> exclusive scan -> stable scatter.  Ranks inside a warp
-// come from __match_any_sync peer masks, ranks across warps from a per-warp
+// come from peer masks (one ballot per bit of the expert id), ranks across warps from a per-warp
 // count table and a column scan, ranks across CTAs from a per-chunk count table
-// that every scatter CTA reads whole, so the result (ascending expanded id inside every expert)
-// never depends on atomic ordering.  No kernel waits on another CTA.
+// whose columns are scanned over the chunks, so the result (ascending expanded id
+// inside every expert) never depends on atomic ordering.  Up to kSmallRows rows
+// one CTA does it all; beyond, one launch of at most one CTA per SM does it in
+// three phases separated by two grid barriers (bounded waits).
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -246,27 +248,29 @@ __device__ __forceinline__ void warp_route_token(const float* __restrict__ row, 
     warp_select_token<V, VEC>(v, E, k, lane, ids, weights, ids_s, cand);
 }
 
-// Thread e (< E) owns expert e with `count` rows at permuted offset `off` and
-// writes its tiles: as few as ceil(count / nt) allows, of near-equal size rounded
-// to the MMA's 16-column granule (so no tile is a short tail that streams a whole
-// weight block for a few rows), the last one taking the remainder.
-__device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int count, int off,
-                                                      const PermuteAux& aux, int* sums)
+// The tiles of an expert with `count` rows: as few as ceil(count / nt) allows, of
+// near-equal size q rounded to the MMA's 16-column granule (so no tile is a short
+// tail that streams a whole weight block for a few rows), the last one taking the
+// remainder.  Returns the tile count (0 for an empty expert).
+__device__ __forceinline__ int expert_tile_count(int count, int nt, int& q)
 {
-    int n = 0, q = aux.nt;
-    if (owns && count > 0) {
-        const int n0 = (count + aux.nt - 1) / aux.nt;
-        const int even = (count + n0 - 1) / n0;
-        q = min(aux.nt, (even + 15) & ~15);
-        n = (count + q - 1) / q;
-    }
-    int total;
-    const int start = block_exclusive_scan(n, sums, total);
+    q = nt;
+    if (count <= 0) return 0;
+    const int n0 = (count + nt - 1) / nt;
+    const int even = (count + n0 - 1) / n0;
+    q = min(nt, (even + 15) & ~15);
+    return (count + q - 1) / q;
+}
+
+// Writes expert e's n tiles (size q, the expert's rows from permuted offset
+// `off`) at tile index `start`.
+__device__ __forceinline__ void write_expert_tiles(int e, int count, int off, int n, int q,
+                                                   int start, const PermuteAux& aux)
+{
     // debug build: never past the tile array (only out-of-contract offsets can
     // ask for more tiles than it holds)
     if (n > 0 && !debug_in_range(start + n - 1, 0, aux.max_tiles, aux.err))
         n = max(0, aux.max_tiles - start);
-    if (kDebugChecks) total = min(total, aux.max_tiles);
     for (int i = 0; i < n; ++i) {
         Tile t;
         t.expert = e;
@@ -277,44 +281,94 @@ __device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int coun
         t.pad[0] = t.pad[1] = t.pad[2] = 0;
         aux.tiles[start + i] = t;
     }
+}
+
+// Thread e (< E) owns expert e with `count` rows at permuted offset `off` and
+// writes its tiles; thread 0 writes the tile count.
+__device__ __forceinline__ void write_tiles_and_reset(bool owns, int e, int count, int off,
+                                                      const PermuteAux& aux, int* sums)
+{
+    int q;
+    const int n = owns ? expert_tile_count(count, aux.nt, q) : 0;
+    int total;
+    const int start = block_exclusive_scan(n, sums, total);
+    if (kDebugChecks) total = min(total, aux.max_tiles);
+    if (n > 0) write_expert_tiles(e, count, off, n, q, start, aux);
     if (threadIdx.x == 0) *aux.num_tiles = total;
 }
 
-// Per-warp histogram of rows [r0, r1) of ids_s into table[warp*E + e].
-__device__ __forceinline__ void warp_count(const int* ids_s, int r0, int r1, int* table_row)
+// Expert ids of a range of rows: staged in shared memory, or read from global
+// memory (the debug build redirects an out-of-range id to expert 0 on each read).
+struct StagedIds {
+    const int* s;
+    __device__ __forceinline__ int operator()(int r) const { return s[r]; }
+};
+struct GlobalIds {
+    const int32_t* g;
+    int E;
+    int32_t* err;
+    __device__ __forceinline__ int operator()(int r) const
+    {
+        const int id = g[r];
+        return debug_in_range(id, 0, E, err) ? id : 0;
+    }
+};
+
+// Bits of an expert id below E (0 for E = 1).
+__device__ __forceinline__ int expert_bits(int E) { return E <= 1 ? 0 : 32 - __clz(E - 1); }
+
+// Mask of the valid lanes whose key equals this lane's key e (in [0, 2^nbits),
+// nbits <= 10).  Up to 16 experts: __match_any_sync, whose cost grows with the
+// number of distinct keys in the warp.  Beyond: one ballot per key bit (two keys
+// are equal exactly when they agree on every bit), a constant cost, lower than
+// __match_any_sync's once a warp holds many distinct experts.
+__device__ __forceinline__ unsigned warp_peers(int e, bool valid, int nbits)
+{
+    if (nbits <= 4) {
+        const unsigned vm = __ballot_sync(kFull, valid);
+        return valid ? __match_any_sync(vm, e) : 0u;
+    }
+    unsigned peers = __ballot_sync(kFull, valid);
+    for (int b = 0; b < nbits; ++b) {
+        const bool bit = (e >> b) & 1;
+        const unsigned m = __ballot_sync(kFull, bit);
+        peers &= bit ? m : ~m;
+    }
+    return peers;
+}
+
+// Per-warp histogram of rows [r0, r1) into table_row[e] (ids below 2^nbits).
+template <typename Ids>
+__device__ __forceinline__ void warp_count(const Ids& id_at, int r0, int r1, int* table_row,
+                                           int nbits)
 {
     const int lane = threadIdx.x & 31;
     for (int base = r0; base < r1; base += 32) {
         const int r = base + lane;
         const bool valid = r < r1;
-        const int e = valid ? ids_s[r] : -1;
-        const unsigned vm = __ballot_sync(kFull, valid);
-        if (valid) {
-            const unsigned peers = __match_any_sync(vm, e);
-            if (lane == __ffs(peers) - 1) table_row[e] += __popc(peers);
-        }
+        const int e = valid ? id_at(r) : 0;
+        const unsigned peers = warp_peers(e, valid, nbits);
+        if (valid && lane == __ffs(peers) - 1) table_row[e] += __popc(peers);
         __syncwarp();
     }
 }
 
-// Stable scatter of rows [r0, r1): table_row[e] holds the absolute position of
-// the next row of expert e owned by this warp.
-__device__ __forceinline__ void warp_scatter(const int* ids_s, int r0, int r1, int id_base,
-                                             int* table_row, int32_t* __restrict__ rows_out)
+// Stable scatter of rows [r0, r1): the next row of expert e owned by this warp
+// goes to position (base ? base[e] : 0) + table_row[e].
+template <typename Ids>
+__device__ __forceinline__ void warp_scatter(const Ids& id_at, int r0, int r1, int id_base,
+                                             const int* base, int* table_row,
+                                             int32_t* __restrict__ rows_out, int nbits)
 {
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
-    for (int base = r0; base < r1; base += 32) {
-        const int r = base + lane;
+    for (int b = r0; b < r1; b += 32) {
+        const int r = b + lane;
         const bool valid = r < r1;
-        const int e = valid ? ids_s[r] : -1;
-        const unsigned vm = __ballot_sync(kFull, valid);
-        unsigned peers = 0;
+        const int e = valid ? id_at(r) : 0;
+        const unsigned peers = warp_peers(e, valid, nbits);
         int pos = 0;
-        if (valid) {
-            peers = __match_any_sync(vm, e);
-            pos = table_row[e] + __popc(peers & lt);
-        }
+        if (valid) pos = (base ? base[e] : 0) + table_row[e] + __popc(peers & lt);
         __syncwarp();
         if (valid) {
             rows_out[pos] = id_base + r;
@@ -451,7 +505,7 @@ __global__ void __launch_bounds__(1024, 1)
 
     const int per_warp = (R + W - 1) / W;
     const int r0 = min(R, warp * per_warp), r1 = warp < W ? min(R, r0 + per_warp) : r0;
-    if (warp < W) warp_count(ids_s, r0, r1, table + warp * E);
+    if (warp < W) warp_count(StagedIds{ids_s}, r0, r1, table + warp * E, expert_bits(E));
     __syncthreads();
 
     const bool owns = threadIdx.x < E;
@@ -473,120 +527,218 @@ __global__ void __launch_bounds__(1024, 1)
     write_tiles_and_reset(owns, e, cnt, off, aux, sums);
     __syncthreads();
 
-    if (warp < W) warp_scatter(ids_s, r0, r1, 0, table + warp * E, rows_out);
+    if (warp < W)
+        warp_scatter(StagedIds{ids_s}, r0, r1, 0, nullptr, table + warp * E, rows_out,
+                     expert_bits(E));
 }
 
-__global__ void __launch_bounds__(1024) chunk_count_kernel(const int32_t* __restrict__ ids, int R,
-                                                           int E, int32_t* __restrict__ counts,
-                                                           int32_t* err)
-{
-    extern __shared__ int hist[];
-    pdl_wait();
-    pdl_launch_dependents();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-    __syncthreads();
-    const int r0 = blockIdx.x * kChunkRows, r1 = min(R, r0 + kChunkRows);
-    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
-        const int e = ids[r];
-        atomicAdd(&hist[debug_in_range(e, 0, E, err) ? e : 0], 1);
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = hist[e];
-}
+// ------------------------------------------- one-launch multi-CTA permutation
 
-// After chunk_count_kernel, for experts 32 b .. 32 b + 31 (CTA b, lane = expert):
-// warp w walks the chunks [w L, (w + 1) L) (L = ceil(n_chunks / 32)) of its
-// expert, the 32 warps' sums are scanned in shared memory, and counts[c][e] is
-// overwritten with P[c][e] = the rows of e in the chunks before c.  Row n_chunks
-// of the table receives the expert's total.  Every chunk read is coalesced over
-// the 32 experts of a warp.
-__global__ void __launch_bounds__(1024, 1)
-    chunk_prefix_kernel(int32_t* __restrict__ counts, int n_chunks, int E)
+constexpr int kPermWarps = 32;         // warps per CTA
+constexpr int kPermRankWarps = 8;      // of which rank the chunk, one contiguous piece each
+constexpr int kPermStageRows = 8192;   // chunks up to this many rows are staged in shared memory
+constexpr int kPermMaxChunks = 256;    // grid bound (the prefix phase's chunks per lane <= 8)
+constexpr int kPermLaneChunks = kPermMaxChunks / 32;
+
+// Thread 0 of a CTA: bounded wait (2 s) until `ok()` holds.  Gives up early when
+// another CTA recorded an abort of this call; on its own timeout records the
+// abort and kDeviceErrorMagic in *err.
+template <typename Pred>
+__device__ bool grid_wait(GridBar* bar, unsigned long long gen, int32_t* err, Pred ok)
 {
-    __shared__ int part[32][33];
-    pdl_wait();
-    pdl_launch_dependents();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * 32 + lane;
-    const int L = (n_chunks + 31) / 32;
-    const int c0 = min(n_chunks, warp * L), c1 = min(n_chunks, c0 + L);
-    int sum = 0;
-    if (e < E)
-        for (int c = c0; c < c1; ++c) sum += __ldcg(counts + (size_t)c * E + e);
-    part[warp][lane] = sum;
-    __syncthreads();
-    int pre = 0;
-    for (int w = 0; w < warp; ++w) pre += part[w][lane];
-    if (e < E) {
-        int run = pre;
-        for (int c = c0; c < c1; ++c) {
-            const int v = __ldcg(counts + (size_t)c * E + e);
-            counts[(size_t)c * E + e] = run;
-            run += v;
+    if (ok()) return true;
+    const uint64_t t0 = globaltimer_ns();
+    volatile unsigned long long* abort = &bar->abort;
+    for (;;) {
+        __nanosleep(32);
+        if (ok()) return true;
+        if (*abort == gen) return false;
+        if (globaltimer_ns() - t0 > 2000000000ull) {
+            *abort = gen;
+            atomicExch(err, kDeviceErrorMagic);
+            return false;
         }
-        if (warp == 31) counts[(size_t)n_chunks * E + e] = run;  // the expert's total
     }
 }
 
-constexpr int kRankWarps = 8;
-
-// One CTA per chunk of kChunkRows expanded rows, after chunk_prefix_kernel.  The
-// expert totals (row n_chunks of the table) give expert_offsets by an exclusive
-// scan over experts (CTA 0 also writes them and the tile list); base[e] =
-// expert_offsets[e] + P[chunk][e] is where the chunk's first row of expert e
-// goes.  The chunk's rows are ranked stably with per-warp count tables (a warp's
-// rows in order, warps in order) and scattered.
-__global__ void __launch_bounds__(1024, 1)
-    chunk_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, int n_chunks,
-                         const int32_t* __restrict__ prefix, int32_t* __restrict__ offsets,
-                         int32_t* __restrict__ rows_out, PermuteAux aux)
+// The stable permutation of R > kSmallRows rows in one launch of G CTAs (all
+// resident at once; at most one per SM), CTA c owning the S rows from c*S (S a
+// multiple of 32).
+//   1. The CTA counts its chunk's experts into counts[c][*] and arrives at the
+//      grid barrier; while the others arrive, each of kPermRankWarps warps counts
+//      its contiguous piece of the chunk, and per expert the pieces' counts
+//      become exclusive prefixes over the pieces.
+//   2. After the barrier, warp w of CTA c takes experts e = w G + c, ...: its
+//      lanes split the G chunks into contiguous runs, and the warp turns column
+//      e of the table into exclusive prefixes over the chunks (in place) with the
+//      expert's total in row G.  Second barrier.
+//   3. Every CTA scans the totals (and the experts' tile counts) into expert
+//      offsets (and first tiles); CTA c writes the offsets and tiles of experts
+//      c, c + G, ...  Then each of the kPermRankWarps warps places its piece in
+//      order: row r of expert e goes to offset[e] + rows of e in earlier chunks +
+//      rows of e in earlier pieces + rows of e before r in the piece (peer masks).
+// A chunk too large to stage in shared memory (STAGED false) is read from global
+// memory both times.
+template <bool STAGED>
+__global__ void __launch_bounds__(kPermWarps * 32, 1)
+    grid_permute_kernel(const int32_t* __restrict__ ids, int R, int E, int S,
+                        int32_t* __restrict__ offsets, int32_t* __restrict__ rows_out,
+                        PermuteAux aux)
 {
     extern __shared__ int smem[];
-    __shared__ int sums[32];
-    int* ids_s = smem;                 // kChunkRows
-    int* table = smem + kChunkRows;    // [kRankWarps][E]
-    const int warp = threadIdx.x >> 5;
+    __shared__ int2 sums2[32];
+    __shared__ int go;
+    int* table = smem;                      // [kPermRankWarps][E]
+    int* hist = smem + kPermRankWarps * E;  // [E]: the chunk's counts, later its bases
+    int* ids_s = smem + ((kPermRankWarps * E + E + 3) & ~3);  // [S] when STAGED (16-byte aligned)
+    const int G = gridDim.x, c = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    GridBar* bar = aux.bar;
+    int32_t* counts = aux.chunk_counts;
+    const unsigned long long gen = aux.gen;
     pdl_wait();
     pdl_launch_dependents();
-    const int c0 = blockIdx.x * kChunkRows, n = min(kChunkRows, R - c0);
-    const bool owns = threadIdx.x < E;
-    const int e = threadIdx.x;
-    // the three loads are independent: issue them before anything waits
-    const int total_e = owns ? __ldcg(prefix + (size_t)n_chunks * E + e) : 0;
-    const int pre_e = owns ? __ldcg(prefix + (size_t)blockIdx.x * E + e) : 0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int id = ids[c0 + i];
-        ids_s[i] = debug_in_range(id, 0, E, aux.err) ? id : 0;
+    if (c == 0 && threadIdx.x == 0) {  // this call's barrier count starts at 0
+        bar->count = 0;
+        __threadfence();
+        st_release_gpu_u64(&bar->gen, gen);
     }
-    for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) table[i] = 0;
-    int total;
-    const int off = block_exclusive_scan(total_e, sums, total);  // ends with a barrier
-    if (blockIdx.x == 0) {
-        if (owns) offsets[e] = off;
-        if (threadIdx.x == 0) offsets[E] = total;
-        write_tiles_and_reset(owns, e, total_e, off, aux, sums);
+    const int c0 = c * S, n = min(S, R - c0);
+    for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < kPermRankWarps * E / 4; i += blockDim.x)
+        reinterpret_cast<int4*>(table)[i] = make_int4(0, 0, 0, 0);
+    if (STAGED) {
+        // 16-byte loads, all in flight before any store (c0 is a multiple of 32,
+        // so ids + c0 keeps the 16-byte alignment of ids)
+        constexpr int kVec = kPermStageRows / 4 / (kPermWarps * 32);
+        const int4* src = reinterpret_cast<const int4*>(ids + c0);
+        int4 v[kVec];
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const int i = (threadIdx.x + j * kPermWarps * 32) * 4;
+            v[j] = i + 3 < n ? src[i / 4] : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const int i = (threadIdx.x + j * kPermWarps * 32) * 4;
+            if (i + 3 < n) reinterpret_cast<int4*>(ids_s)[i / 4] = v[j];
+        }
+        const int tail = n & ~3;  // the last n % 4 rows
+        if (threadIdx.x < n - tail) ids_s[tail + threadIdx.x] = ids[c0 + tail + threadIdx.x];
     }
-
-    // kRankWarps warps rank the chunk's rows, kChunkRows / kRankWarps each, in
-    // order: fewer count rows to clear and to scan than one per warp of the CTA
-    constexpr int per_warp = kChunkRows / kRankWarps;
-    const int r0 = min(n, warp * per_warp), r1 = min(n, r0 + per_warp);
-    if (warp < kRankWarps) warp_count(ids_s, r0, r1, table + warp * E);
     __syncthreads();
-    if (owns) {
-        // the ranking warps' counts of expert e, read before any is overwritten
-        int v[kRankWarps];
+
+    // 1. the chunk's counts
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        int id = STAGED ? ids_s[i] : ids[c0 + i];
+        if (!debug_in_range(id, 0, E, aux.err)) id = 0;
+        if (STAGED) ids_s[i] = id;
+        atomicAdd(&hist[id], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += blockDim.x) counts[(size_t)c * E + i] = hist[i];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        go = grid_wait(bar, gen, aux.err,
+                       [&] { return ld_acquire_gpu_u64(&bar->gen) == gen; });
+        if (go) red_release_gpu_add(reinterpret_cast<int*>(&bar->count), 1);
+    }
+    // the pieces' counts while the other CTAs arrive
+    const int nbits = expert_bits(E);
+    const int per = (n + kPermRankWarps - 1) / kPermRankWarps;
+    const int r0 = min(n, warp * per), r1 = warp < kPermRankWarps ? min(n, r0 + per) : r0;
+    if (STAGED)
+        warp_count(StagedIds{ids_s}, r0, r1, table + warp * E, nbits);
+    else
+        warp_count(GlobalIds{ids + c0, E, aux.err}, r0, r1, table + warp * E, nbits);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int v[kPermRankWarps];
 #pragma unroll
-        for (int w = 0; w < kRankWarps; ++w) v[w] = table[w * E + e];
-        int run = off + pre_e;
+        for (int w = 0; w < kPermRankWarps; ++w) v[w] = table[w * E + e];
+        int run = 0;
 #pragma unroll
-        for (int w = 0; w < kRankWarps; ++w) {
+        for (int w = 0; w < kPermRankWarps; ++w) {
             table[w * E + e] = run;
             run += v[w];
         }
     }
+    if (threadIdx.x == 0 && go)
+        go = grid_wait(bar, gen, aux.err, [&] {
+            return (uint32_t)ld_acquire_gpu(reinterpret_cast<const int*>(&bar->count)) >= (uint32_t)G;
+        });
     __syncthreads();
-    if (warp < kRankWarps) warp_scatter(ids_s, r0, r1, c0, table + warp * E, rows_out);
+    if (!go) return;
+
+    // 2. per expert: exclusive prefixes over the chunks, and the total
+    {
+        const int L = (G + 31) / 32;
+        const int cb = min(G, lane * L), ce = min(G, cb + L);
+        for (int e = warp * G + c; e < E; e += kPermWarps * G) {
+            int v[kPermLaneChunks];
+#pragma unroll
+            for (int i = 0; i < kPermLaneChunks; ++i)  // all loads in flight at once
+                v[i] = __ldcg(counts + (size_t)min(cb + i, G - 1) * E + e);
+            int sum = 0;
+#pragma unroll
+            for (int i = 0; i < kPermLaneChunks; ++i) {
+                if (cb + i >= ce) v[i] = 0;
+                sum += v[i];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += t;
+            }
+            int run = incl - sum;
+#pragma unroll
+            for (int i = 0; i < kPermLaneChunks; ++i)
+                if (cb + i < ce) {
+                    counts[(size_t)(cb + i) * E + e] = run;
+                    run += v[i];
+                }
+            if (lane == 31) counts[(size_t)G * E + e] = incl;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        red_release_gpu_add(reinterpret_cast<int*>(&bar->count), 1);
+        go = grid_wait(bar, gen, aux.err, [&] {
+            return (uint32_t)ld_acquire_gpu(reinterpret_cast<const int*>(&bar->count)) >=
+                   2u * (uint32_t)G;
+        });
+    }
+    __syncthreads();
+    if (!go) return;
+
+    // 3. offsets and tiles, the chunk's bases, the placement
+    const bool owns = threadIdx.x < E;
+    const int e = threadIdx.x;
+    const int total_e = owns ? __ldcg(counts + (size_t)G * E + e) : 0;
+    const int pre_e = owns ? __ldcg(counts + (size_t)c * E + e) : 0;
+    int q = 0;
+    const int nt_e = owns ? expert_tile_count(total_e, aux.nt, q) : 0;
+    int2 tot;
+    const int2 ex = block_exclusive_scan2(make_int2(total_e, nt_e), sums2, tot);  // ends with a barrier
+    if (owns) {
+        hist[e] = ex.x + pre_e;
+        if (e % G == c) {  // this CTA publishes expert e
+            offsets[e] = ex.x;
+            write_expert_tiles(e, total_e, ex.x, nt_e, q, ex.y, aux);
+        }
+    }
+    if (c == 0 && threadIdx.x == 0) {
+        offsets[E] = tot.x;
+        *aux.num_tiles = kDebugChecks ? min(tot.y, aux.max_tiles) : tot.y;
+    }
+    __syncthreads();
+    if (STAGED) {
+        warp_scatter(StagedIds{ids_s}, r0, r1, c0, hist, table + warp * E, rows_out, nbits);
+    } else {
+        warp_scatter(GlobalIds{ids + c0, E, aux.err}, r0, r1, c0, hist, table + warp * E,
+                     rows_out, nbits);
+    }
 }
 
 __global__ void __launch_bounds__(1024) build_tiles_kernel(const int32_t* __restrict__ offsets,
@@ -698,25 +850,28 @@ cudaError_t launch_small_route_permute(const float* logits, int T, int E, int k,
 #undef MOE_SMALL
 }
 
-size_t large_permute_smem(int E) { return sizeof(int) * (size_t)(kChunkRows + kRankWarps * E); }
-
 cudaError_t launch_large_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                                  int32_t* rows, const PermuteAux& aux, cudaStream_t st)
 {
-    const int R = T * k;
-    const int n_chunks = (R + kChunkRows - 1) / kChunkRows;
-    cudaError_t err = launch(chunk_count_kernel, dim3(n_chunks), dim3(1024), sizeof(int) * E, st,
-                             ids, R, E, aux.chunk_counts, aux.err);
-    if (err != cudaSuccess) return err;
-    err = launch(chunk_prefix_kernel, dim3((E + 31) / 32), dim3(1024), 0, st, aux.chunk_counts,
-                 n_chunks, E);
-    if (err != cudaSuccess) return err;
-    const size_t smem = large_permute_smem(E);
-    err = cudaFuncSetAttribute(chunk_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-    if (err != cudaSuccess) return err;
-    return launch(chunk_scatter_kernel, dim3(n_chunks), dim3(1024), smem, st, ids, R, E, n_chunks,
-                  (const int32_t*)aux.chunk_counts, offsets, rows, aux);
+    const long long R = (long long)T * k;
+    int gmax = device_sms();
+    if (gmax > aux.max_chunks) gmax = aux.max_chunks;
+    if (gmax > kPermMaxChunks) gmax = kPermMaxChunks;
+    if (gmax < 1) return cudaErrorInvalidValue;
+    // rows per chunk: a multiple of 32, and as few chunks as that leaves
+    const long long S = (((R + gmax - 1) / gmax) + 31) & ~31LL;
+    const int G = (int)((R + S - 1) / S);
+    const bool staged = S <= kPermStageRows;
+    const size_t smem =
+        sizeof(int) * ((((size_t)kPermRankWarps * E + E + 3) & ~(size_t)3) + (staged ? (size_t)S : 0));
+    auto go = [&](auto kern) {
+        cudaError_t err =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        return launch(kern, dim3(G), dim3(kPermWarps * 32), smem, st, ids, (int)R, E, (int)S,
+                      offsets, rows, aux);
+    };
+    return staged ? go(grid_permute_kernel<true>) : go(grid_permute_kernel<false>);
 }
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int R, const PermuteAux& aux,
