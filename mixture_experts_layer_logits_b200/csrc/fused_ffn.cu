@@ -153,9 +153,9 @@ using FCfg = Cfg<0, NT, kFusedReserve>;
 // then staging, Aux and the unit table as in the bf16 kernel.  A unit's K range
 // is always an even number of K tiles (H and I are multiples of 128, w2 slices
 // are rounded up to even lengths), so a pair stage never straddles two units.
-// Tensor memory (all 512 columns): accumulators in [0, 256), kSA converted A
-// stages in [256, 512), each two 128 x 64 bf16 tiles (row = lane, bf16 pairs
-// along 32 columns per tile).  Aux's barrier arrays are shared out in the order
+// Tensor memory (all 512 columns): kNBuf accumulators from column 0, then kSA
+// converted A stages up to column 512, each two 128 x 64 bf16 tiles (row = lane,
+// bf16 pairs along 32 columns per tile).  Aux's barrier arrays are shared out in the order
 // A8, A, B.
 template <int NT>
 struct W8Cfg {
@@ -164,19 +164,24 @@ struct W8Cfg {
     static constexpr int kBoxBytes = kBM * 2 * kBK;  // one [128 x 128]-byte box
     static constexpr int kBBytes = C::kBTileBytes;
     static constexpr int kTmemCols = 512;
-    static constexpr int kNBuf = 256 / C::kAccCols;  // accumulator buffers: 8, 4, 2
-    static constexpr int kACol0 = 256;
+    // accumulator buffers: 4 at NT = 16, else 2 (a decode unit streams many K
+    // tiles, so two buffers keep the MMA a unit ahead of the epilogue); the rest
+    // of tensor memory holds converted A stages: 6 at NT <= 32, 4 at NT = 64
+    static constexpr int kNBuf = C::kAccCols <= 32 ? 4 : 2;
+    static constexpr int kACol0 = kNBuf * C::kAccCols;
     static constexpr int kACols = 2 * kBK / 2;       // columns per converted stage
-    static constexpr int kSA = 256 / kACols;
+    static constexpr int kSA = ((512 - kACol0) / kACols) & ~1;
     static constexpr int kSB = NT <= 32 ? 6 : 4;
     // The MMA frees A and B slots two K tiles at a time (one tcgen05.commit per
     // pair: each commit drains the tensor pipe, about 200-300 cycles, as much as
     // four of these M = 128, N <= 64 MMAs cost), so both rings have even depth
-    // and their "empty" barriers are per slot pair.
+    // and their "empty" barriers are per slot pair.  When both rings have the same
+    // depth, one commit frees both: the converters and the token-operand warp wait
+    // on the A ring's barrier.
     static_assert(kSA % 2 == 0 && kSB % 2 == 0, "slot pairs");
     static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kFusedReserve;
     static constexpr int kS8Raw = (C::kMaxSmem - kFixed - kSB * kBBytes) / kA8Bytes;
-    static constexpr int kS8 = kS8Raw < 16 - kSA - kSB ? kS8Raw : 16 - kSA - kSB;
+    static constexpr int kS8 = kS8Raw < kBarSlots - kSA - kSB ? kS8Raw : kBarSlots - kSA - kSB;
     static constexpr int kRingBytes = kSB * kBBytes + kS8 * kA8Bytes;
     static constexpr int kSmemBytes = kFixed + kRingBytes;
     static constexpr int kPf = 2;  // pair stages the producer prefetches into L2 ahead
@@ -188,7 +193,8 @@ struct W8Cfg {
     static constexpr int kConv0 = 4, kConvExtra0 = 16, kConvWarps = 8;
     // barrier slots in Aux's full/empty arrays
     static constexpr int kBar8 = 0, kBarA = kS8, kBarB = kS8 + kSA;
-    static_assert(kS8 >= 3 && kS8 + kSA + kSB <= 16, "barrier slots");
+    static constexpr int kEmptyB = kSA == kSB ? kBarA : kBarB;  // the B ring's "empty" barriers
+    static_assert(kS8 >= 3 && kS8 + kSA + kSB <= kBarSlots, "barrier slots");
     static_assert(kSmemBytes <= C::kMaxSmem, "shared memory");
     static_assert(kACol0 + kSA * kACols <= kTmemCols && kNBuf * C::kAccCols <= kACol0, "TMEM");
 };
@@ -783,7 +789,8 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                     if constexpr (W8) {  // free the A and B slot pairs when read
                         if (q & 1) {
                             umma_commit(&aux->empty[R8::kBarA + (q >> 1) % (R8::kSA / 2)]);
-                            umma_commit(&aux->empty[R8::kBarB + (q >> 1) % (R8::kSB / 2)]);
+                            if constexpr (R8::kSA != R8::kSB)
+                                umma_commit(&aux->empty[R8::kBarB + (q >> 1) % (R8::kSB / 2)]);
                         }
                         ++q;
                     } else {
@@ -843,7 +850,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 const int sb = q % R8::kSB, pb = (q >> 1) % (R8::kSB / 2);
                 uint64_t* fb = &aux->full[R8::kBarB + sb];
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(&aux->empty[R8::kBarB + pb],
+                                mbar_wait(&aux->empty[R8::kEmptyB + pb],
                                           (uint32_t)((((q >> 1) / (R8::kSB / 2)) & 1) ^ 1),
                                           abort_flag))) {
                     if (lane == 0) flag_error(a.err, aux);

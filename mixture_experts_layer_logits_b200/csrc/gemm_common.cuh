@@ -64,9 +64,11 @@ struct Cfg {
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
 };
 
+constexpr int kBarSlots = 20;  // ring barriers in Aux
+
 struct Aux {
-    uint64_t full[16];
-    uint64_t empty[16];
+    uint64_t full[kBarSlots];
+    uint64_t empty[kBarSlots];
     uint64_t tfull[8];
     uint64_t tempty[8];
     uint64_t drain;

@@ -82,6 +82,20 @@ def test_route_adversarial_ties(E, k):
     assert_routing_equal(ids, wts, ref_ids, ref_w)
 
 
+@pytest.mark.parametrize("T,E,k", [(63, 1024, 16), (63, 1000, 8), (7, 512, 8), (33, 300, 16),
+                                   (5, 260, 1), (129, 772, 4)])
+def test_route_many_experts_odd_counts(T, E, k):
+    """256 < E <= 1024 (the streaming router: 16 or 32 values per lane, rows
+    staged in shared memory) with token counts that leave the last CTA partly
+    idle, experts that do not fill the last float4 slots, and ties that push
+    tokens onto the exact path."""
+    logits = adversarial_logits(T, E, seed=T * 7 + E + k)
+    ids, wts = moe.moe_route(logits.cuda(), k)
+    torch.cuda.synchronize()
+    ref_ids, ref_w = oracle.route(logits.numpy(), k)
+    assert_routing_equal(ids, wts, ref_ids, ref_w)
+
+
 # ------------------------------------------------------------------ permutation
 
 @pytest.mark.parametrize("T,E,k,hot", [(16, 8, 2, False), (8, 128, 8, False), (64, 256, 8, True),
