@@ -57,7 +57,7 @@ NCU_TRAFFIC = {
     ("prefill", "w13"): 3_694_407_168 + 205_702_912,
     ("prefill", "w2"): 1_829_378_048 + 509_899_264,
     ("decode", "fused_ffn"): 509_752_832 + 3_875_328,
-    ("decode+e4m3", "fused_ffn"): 257_118_464 + 3_917_056,
+    ("decode+e4m3", "fused_ffn"): 256_922_368 + 3_352_576,
     ("routing_stress", "route"): 67_143_424 + 793_344,
 }
 
