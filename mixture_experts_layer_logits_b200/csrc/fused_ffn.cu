@@ -648,8 +648,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             uint8_t* const pring = W8 ? ring8 : ring;
             int stage = 0;
             uint32_t phase = 0;
-            int issued[16];
-            for (int s = 0; s < NS; ++s) issued[s] = 0;
+            int fills = 0;  // ring stage fills so far (fill q went to stage q % stages)
             bool ok = true;
             bool counters = false;  // this call's counters are zeroed (wait_counters)
             for (int i = 0; ok; ++i) {
@@ -705,7 +704,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                         tma_prefetch_l2_2d(tm, (kt + 2 * R8::kPf) * kBK, row0);
                         tma_prefetch_l2_2d(tm, (kt + 2 * R8::kPf) * kBK, row1);
                     }
-                    issued[stage] += 1;
+                    ++fills;
                     if (++stage == NS) {
                         stage = 0;
                         phase ^= 1u;
@@ -714,12 +713,14 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             }
             if (!ok || *abort_flag) {
                 // let every TMA load already issued land before the CTA can exit
-                for (int s = 0; s < NS; ++s)
-                    if (issued[s] > 0) {
+                for (int s = 0; s < NS; ++s) {
+                    const int n_s = fills > s ? (fills - s + NS - 1) / NS : 0;  // fills of stage s
+                    if (n_s > 0) {
                         volatile int never = 0;
-                        mbar_wait(&aux->full[s], (uint32_t)((issued[s] - 1) & 1), &never,
+                        mbar_wait(&aux->full[s], (uint32_t)((n_s - 1) & 1), &never,
                                   500000000ull);
                     }
+                }
             }
         }
     } else if (warp == 1) {

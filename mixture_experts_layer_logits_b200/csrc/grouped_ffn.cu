@@ -251,8 +251,7 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
                                                        : l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
-            int issued[16];
-            for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
+            int fills = 0;  // ring stage fills so far (fill q went to stage q % stages)
             bool ok = true;
             bool dep_ready = MODE == 0;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -299,7 +298,7 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
                         tma_prefetch_l2_2d(&tm_w, (kt + kPrefetch) * kBK, row);
                         tma_prefetch_l2_2d(&tm_w, (kt + kPrefetch) * kBK, row1);
                     }
-                    issued[stage] += 1;
+                    ++fills;
                     if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -309,12 +308,15 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
             if (!dep_ready) pdl_wait();  // (no unit here) the grid still depends on it
             if (!ok || *abort_flag) {
                 // let every TMA load already issued land before the CTA can exit
-                for (int s = 0; s < C::kStages; ++s)
-                    if (issued[s] > 0) {
+                for (int s = 0; s < C::kStages; ++s) {
+                    // fills of stage s
+                    const int n_s = fills > s ? (fills - s + C::kStages - 1) / C::kStages : 0;
+                    if (n_s > 0) {
                         volatile int never = 0;
-                        mbar_wait(&aux->full[s], (uint32_t)((issued[s] - 1) & 1), &never,
+                        mbar_wait(&aux->full[s], (uint32_t)((n_s - 1) & 1), &never,
                                   500000000ull);
                     }
+                }
             }
         }
     } else if (warp == 1) {
