@@ -20,8 +20,8 @@ __device__ __forceinline__ bool key_before(float va, int ia, float vb, int ib)
     return va > vb || (va == vb && ia < ib);
 }
 
-// Sorts one (value, index) key per lane across groups of W lanes (W = 16: each
-// half-warp on its own; W = 32: the warp) so that the group's first lane holds
+// Sorts one (value, index) key per lane across groups of W lanes (W = 8 or 16:
+// each group on its own; W = 32: the warp) so that the group's first lane holds
 // the key that ranks first (larger value, then lower index).  Bitonic network with
 // the "ranks before" relation as the order; keys must be distinct (they are:
 // indices are unique).
@@ -82,9 +82,12 @@ __device__ __forceinline__ void sort_candidates(int total, int lane, const float
         ci = __float_as_int(cc.y);
     }
     __syncwarp();  // cand may be rewritten by this warp's next token
-    // usually about k candidates: then lanes 0..15 hold all of them and a
-    // half-warp network (10 stages instead of 15) orders them the same way
-    if (total <= 16)
+    // usually about k candidates: then lanes 0..7 or 0..15 hold all of them and a
+    // network over 8 or 16 lanes (6 or 10 stages instead of 15) orders them the
+    // same way
+    if (total <= 8)
+        warp_sort_keys<8>(cv, ci, lane);
+    else if (total <= 16)
         warp_sort_keys<16>(cv, ci, lane);
     else
         warp_sort_keys<32>(cv, ci, lane);

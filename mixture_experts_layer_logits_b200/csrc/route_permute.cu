@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 3)
 #pragma unroll
             for (int m = 0; m < kPieces; ++m) {
                 const int e = m * 128 + lane * 4;
-                if (e < E)
+                if (FULL || e < E)
                     cp_async_16_hint(smem_u32(my + (slot * kPieces + m) * 32 + lane), row + e, pol);
             }
         }
@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 3)
 #pragma unroll
         for (int m = 0; m < kPieces; ++m) {
             float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-            if (m * 128 + lane * 4 < E) q = my[(slot * kPieces + m) * 32 + lane];
+            if (FULL || m * 128 + lane * 4 < E) q = my[(slot * kPieces + m) * 32 + lane];
             v[4 * m] = q.x;
             v[4 * m + 1] = q.y;
             v[4 * m + 2] = q.z;
