@@ -102,7 +102,10 @@ def test_route_many_experts_odd_counts(T, E, k):
                                        (512, 8, 8, False),      # R = 4096: single-CTA path
                                        (513, 8, 8, False),      # R = 4104: multi-CTA path
                                        (16384, 1024, 8, False), (8192, 128, 8, True),
-                                       (3000, 1, 1, False), (5000, 37, 3, True)])
+                                       (3000, 1, 1, False), (5000, 37, 3, True),
+                                       # > 148 x 8192 rows: chunks too large to stage in
+                                       # shared memory, ids read from global memory twice
+                                       (200000, 64, 8, True)])
 def test_permute_matches_oracle(T, E, k, hot):
     g = torch.Generator().manual_seed(T + E)
     logits = torch.randn(T, E, generator=g)
