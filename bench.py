@@ -54,11 +54,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (workload, kernel).  An entry is removed when its kernel changes, until it is
 # captured again.
 NCU_TRAFFIC = {
-    ("prefill", "w13"): 3_694_407_168 + 205_702_912,
-    ("prefill", "w2"): 1_829_378_048 + 509_899_264,
-    ("decode", "fused_ffn"): 509_752_832 + 3_875_328,
-    ("decode+e4m3", "fused_ffn"): 256_922_368 + 3_352_576,
-    ("routing_stress", "route"): 67_143_424 + 793_344,
+    ("prefill", "w13"): 3_695_239_424 + 205_527_296,
+    ("prefill", "w2"): 1_815_046_656 + 509_628_928,
+    ("decode", "fused_ffn"): 509_756_416 + 3_208_192,
+    ("decode+e4m3", "fused_ffn"): 256_741_888 + 3_032_320,
+    ("routing_stress", "route"): 67_145_728 + 139_776,
 }
 
 # Records added to the default line (workload name, expert weight format).
