@@ -1332,7 +1332,13 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     a.min_kt_per_split = 4;
     a.s13 = b.s13;
     a.s2 = b.s2;
-    const int grid = plan.grid;
+    // no more CTAs than the most units one phase can have: a small layer (tiny: 32
+    // w13 units) would otherwise launch idle CTAs that still set up and route
+    const long long tiles_max = E < R ? E : R;
+    long long units = tiles_max * a.fb13;
+    units = units > tiles_max * a.fb2 * plan.s2_max ? units : tiles_max * a.fb2 * plan.s2_max;
+    units = units > (long long)T * a.fb2 ? units : (long long)T * a.fb2;
+    const int grid = (int)(units < plan.grid ? units : plan.grid);
     switch (plan.nt * 2 + (w8 ? 1 : 0)) {
     case 32: return launch_fused_nt<16, false>(t13, t2, ta, a, grid, st);
     case 64: return launch_fused_nt<32, false>(t13, t2, ta, a, grid, st);
