@@ -134,7 +134,7 @@ moe_status_t moe_combine(const moe_bf16_t* y, const float* topk_weights, moe_sha
  * path) bit for bit where that path leaves w13 unsplit (H < 512), and up to
  * bf16 rounding of the differently ordered sum otherwise.  Either way every
  * wait is bounded (2 s; then moe_device_status reports MOE_ERR_DEVICE_TIMEOUT).
- * Co-residency: that one launch has one CTA per SM, and its CTAs wait for each
+ * Co-residency: that one launch has at most one CTA per SM, and its CTAs wait for each
  * other's rows, so it assumes all of its CTAs run at once.  Kernels on other
  * streams that hold SMs while it starts delay some of its CTAs; the call stays
  * correct as long as they get an SM within the 2 s bound, and otherwise its

@@ -4,7 +4,7 @@
 // With few tokens per expert the layer is a stream of the touched experts'
 // weights.  As separate launches (grouped_ffn.cu, then the SwiGLU finalize, w2
 // and the combine) every boundary costs a ramp, a tail and a dependency hop on
-// the critical path while HBM idles.  Here one CTA per SM walks a single unit
+// the critical path while HBM idles.  Here one CTA per SM (fewer for small layers) walks a single unit
 // list -- every w13 unit, then every w2 unit -- so the w2 weight stream starts as
 // soon as a CTA has issued its last w13 tile; the steps that need other CTAs'
 // results wait on arrival counters instead of a kernel boundary:
@@ -38,7 +38,7 @@
 // of its w13 units before any w2 unit and all of its units before any combine
 // task; a w13 unit depends on nothing but the routing, a w2 unit only on w13
 // units, a combine task only on w2 units, and within a CTA the epilogue finishes
-// each unit without waiting for a later one.  The grid is one CTA per SM, so
+// each unit without waiting for a later one.  The grid is at most one CTA per SM, so
 // every CTA is resident.  Every wait is bounded (2 s) and also gives up when
 // another CTA has recorded an error.
 //
