@@ -4,10 +4,11 @@
 // With few tokens per expert the layer is a stream of the touched experts'
 // weights.  As separate launches (grouped_ffn.cu, then the SwiGLU finalize, w2
 // and the combine) every boundary costs a ramp, a tail and a dependency hop on
-// the critical path while HBM idles.  Here one CTA per SM (fewer for small layers) walks a single unit
-// list -- every w13 unit, then every w2 unit -- so the w2 weight stream starts as
-// soon as a CTA has issued its last w13 tile; the steps that need other CTAs'
-// results wait on arrival counters instead of a kernel boundary:
+// the critical path while HBM idles.  Here one CTA per SM (fewer for small
+// layers) walks a single unit list -- every w13 unit, then every w2 unit -- so
+// the w2 weight stream starts as soon as a CTA has issued its last w13 tile; the
+// steps that need other CTAs' results wait on arrival counters instead of a
+// kernel boundary:
 //
 //   w13 runs unsplit (one unit = a whole K range), so its epilogue finishes act
 //   itself: bf16(silu(gate) * up).  w2 tile t reads the act rows of tile t,
