@@ -57,7 +57,8 @@ NCU_TRAFFIC = {
     ("prefill", "w13"): 3_695_239_424 + 205_527_296,
     ("prefill", "w2"): 1_815_046_656 + 509_628_928,
     ("decode", "fused_ffn"): 509_756_416 + 3_208_192,
-    ("decode+e4m3", "fused_ffn"): 256_741_888 + 3_032_320,
+    ("decode+e4m3", "fused_ffn"): 256_564_480 + 3_503_616,
+    ("skewed_decode+e4m3", "fused_ffn"): 1_074_733_312 + 8_154_112,
     ("routing_stress", "route"): 67_145_728 + 139_776,
 }
 

@@ -194,13 +194,18 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, moe_shape_t shape,
  * w13_scale fp32 [E, 2I] and w2_scale fp32 [E, H] one scale per weight row:
  * weight (e, r, c) = e4m3(code) * scale(e, r).  Everything else -- arguments,
  * outputs, workspace (moe_workspace_size), routing, roundings, error reporting
- * -- is moe_forward's.  The weights stream at one byte each and are widened to
- * bf16 exactly on chip (into tensor memory, the MMA's A operand), so the
- * tensor-core products are those of the bf16 path; each weight row's scale
- * multiplies its fp32 accumulator row.  Runs
- * only as the one-launch layer (moe_forward_w8_supported; 1 kernel):
+ * -- is moe_forward's.  The weights stream at one byte each and the tensor
+ * cores multiply the codes as they are (E4M3 MMAs).  The other operand, each
+ * token row (x for w13, the bf16 act for w2), is made E4M3 without loss: it is
+ * scaled by a power of two chosen from its largest magnitude and written as two
+ * E4M3 terms that sum to it exactly (entries smaller than 2^-9 of the row's
+ * largest to within 2^-17 of it).  E4M3 products are exact in fp32, so the
+ * accumulators hold the bf16 products; the power of two is undone and each
+ * weight row's scale multiplies its fp32 accumulator row.  Runs only as the
+ * one-launch layer (moe_forward_w8_supported; 1 kernel):
  * MOE_ERR_UNSUPPORTED_SHAPE otherwise, whatever MOE_DISABLE_FUSED says.  Codes
- * 0x7F / 0xFF (NaN) propagate as NaN.  All pointers 16-byte aligned. */
+ * 0x7F / 0xFF (NaN) propagate as NaN; a token whose x row holds an inf or a NaN
+ * gets NaN outputs.  All pointers 16-byte aligned. */
 moe_status_t moe_forward_w8(const moe_bf16_t* x, const float* logits, const uint8_t* w13,
                             const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                             moe_shape_t shape, moe_bf16_t* out, int32_t* topk_ids,

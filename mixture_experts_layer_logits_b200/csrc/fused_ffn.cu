@@ -48,20 +48,22 @@
 // gather (x rows for w13, act tiles for w2), warps 8-15 two epilogue groups,
 // then together the combine.
 //
-// FP8 weights (W8): w13 and w2 arrive as E4M3 codes with one fp32 scale per
+// FP8 weights (F8): w13 and w2 arrive as E4M3 codes with one fp32 scale per
 // weight row (weight = e4m3(q) * scale).  The producer streams the codes -- half
-// the bytes -- into their own ring, one [128 rows x 128 bytes] box per weight
-// block for every two K tiles.  Eight converter warps (warps 4-7 and four extra
-// warps 16-19, 640 threads) widen each K tile to bf16 -- exact, every E4M3 value
-// is a bf16 value -- and store it straight into tensor memory, where the
-// kind::f16 MMA takes its A operand (tcgen05.mma with A in TMEM).  That keeps
-// the bf16 tiles out of shared memory: no second ring there (its 64 KB go to the
-// code ring) and no shared-memory traffic for them, which the MMA's operand reads
-// and the converters would share.  Warp 2 alone fills
-// the token operand into the B ring, its x-row copies arriving on the stage's
-// barrier as they land (cp.async.mbarrier.arrive) so it never waits on them.
-// The scale of a weight row is constant along K, so the epilogue multiplies
-// the fp32 accumulator row by it.
+// the bytes -- two K tiles (128 codes of each weight row) per ring stage, and the
+// tensor cores take them as they are: kind::f8f6f4 MMAs (K = 32 per instruction,
+// so half as many MMAs per weight byte as bf16 MMAs on widened codes would need)
+// with the token operand in E4M3 too.  The gather warps build that operand
+// exactly: each token row (x for w13, act for w2) is scaled by a power of two
+// from its largest magnitude and split into two E4M3 terms whose sum is the
+// scaled bf16 row; the terms of the tile's rows are the MMA's 2 n columns (n =
+// rows rounded up to 16).  E4M3 products are exact in fp32, so the accumulators
+// hold the bf16 products; the epilogue adds each row's two columns, undoes the
+// power of two and multiplies by the weight row's scale.  The x maxima are
+// published per call by the CTAs' epilogue warps before their first unit (token
+// t by CTA t mod G); w13's epilogue folds each act row's largest magnitude into
+// a counter word (atomic max) before its tile_ready arrival, so w2's operand,
+// which waits for that arrival anyway, finds the maxima complete.
 #include <cuda_fp16.h>
 
 #include "gemm_common.cuh"
@@ -110,8 +112,10 @@ struct FusedArgs {
     unsigned long long gen;       // unique to this call
     int32_t* split_out;           // [2] 1, S2 (CTA 0)
     int32_t* err;
-    const float* s13;             // W8: [E, 2I] w13 row scales
-    const float* s2;              // W8: [E, H] w2 row scales
+    const float* s13;             // F8: [E, 2I] w13 row scales
+    const float* s2;              // F8: [E, H] w2 row scales
+    uint32_t* act_max;            // F8: [R] largest |act| per permuted row (fp32 bits), a counter
+    struct XMax* xmax;            // F8: [T] largest |x| per token, tagged with the call's gen
     int T, E, k, H, I, R;
     int kt13, kt2;                // K tiles: H / 64, I / 64
     int fb13, fb2;                // I / 128 gate/up block pairs; ceil(H / 256) w2 block pairs
@@ -148,74 +152,123 @@ constexpr int kFusedReserve = kUnitTableBytes + (int)sizeof(RouteSmem);
 template <int NT>
 using FCfg = Cfg<0, NT, kFusedReserve>;
 
-// The FP8-weight kernel's buffers.  Shared memory after the 1 KB alignment
-// slack: B (kSB token tiles), then A8 (kS8 pair stages: two [128 x 128]-byte
-// E4M3 boxes in the 128-byte swizzle, K tiles kt and kt + 1, written by TMA);
-// then staging, Aux and the unit table as in the bf16 kernel.  A unit's K range
-// is always an even number of K tiles (H and I are multiples of 128, w2 slices
-// are rounded up to even lengths), so a pair stage never straddles two units.
-// Tensor memory (all 512 columns): kNBuf accumulators from column 0, then kSA
-// converted A stages up to column 512, each two 128 x 64 bf16 tiles (row = lane,
-// bf16 pairs along 32 columns per tile).  Aux's barrier arrays are shared out in the order
-// A8, A, B.
+// The FP8-weight kernel with E4M3 MMAs (F8).  One ring, as in the bf16 kernel, each
+// stage two [128 x 128]-byte E4M3 code boxes (TMA; K tiles kt and kt + 1) and
+// the E4M3 token operand of the same 128 K elements: up to 2 NT rows of 128
+// bytes in the 128-byte swizzle, rows [0, n) the hi terms and [n, 2n) the lo
+// terms of the tile's rows (n = rows rounded up to 16), written by the gather
+// warps.  Tensor memory: kNBuf accumulators of 4 NT columns, box 0 (gate block,
+// or the first w2 row block) at column 0 (hi terms in [0, n), lo in [n, 2n)),
+// box 1 at column 2 NT.  After the routing tables, one fp32 row scale per row
+// of the tile for each gather warp.
 template <int NT>
-struct W8Cfg {
+struct F8Cfg {
     using C = FCfg<NT>;
-    static constexpr int kA8Bytes = 2 * kBM * 2 * kBK;
-    static constexpr int kBoxBytes = kBM * 2 * kBK;  // one [128 x 128]-byte box
-    static constexpr int kBBytes = C::kBTileBytes;
+    static constexpr int kBoxBytes = kBM * 2 * kBK;  // [128 rows x 128 codes]
+    static constexpr int kABytes = 2 * kBoxBytes;
+    static constexpr int kBBytes = 2 * NT * 2 * kBK;  // 2 NT rows x 128 codes
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kScaleBytes = kGatherWarps * NT * 4;
+    static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kFusedReserve + kScaleBytes;
+    static constexpr int kStagesRaw = (C::kMaxSmem - kFixed) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kG = kGatherWarps < kStages ? kGatherWarps : kStages;
+    static constexpr int kW = kGatherWarps / kG;
+    static constexpr int kAccCols = 4 * NT;
+    static constexpr int kNBufRaw = 512 / kAccCols;
+    static constexpr int kNBuf = kNBufRaw > 8 ? 8 : kNBufRaw;
     static constexpr int kTmemCols = 512;
-    // accumulator buffers: 4 at NT = 16, else 2 (a decode unit streams many K
-    // tiles, so two buffers keep the MMA a unit ahead of the epilogue); the rest
-    // of tensor memory holds converted A stages: 6 at NT <= 32, 4 at NT = 64
-    static constexpr int kNBuf = C::kAccCols <= 32 ? 4 : 2;
-    static constexpr int kACol0 = kNBuf * C::kAccCols;
-    static constexpr int kACols = 2 * kBK / 2;       // columns per converted stage
-    static constexpr int kSA = ((512 - kACol0) / kACols) & ~1;
-    static constexpr int kSB = NT <= 32 ? 6 : 4;
-    // The MMA frees A and B slots two K tiles at a time (one tcgen05.commit per
-    // pair: each commit drains the tensor pipe, about 200-300 cycles, as much as
-    // four of these M = 128, N <= 64 MMAs cost), so both rings have even depth
-    // and their "empty" barriers are per slot pair.  When both rings have the same
-    // depth, one commit frees both: the converters and the token-operand warp wait
-    // on the A ring's barrier.
-    static_assert(kSA % 2 == 0 && kSB % 2 == 0, "slot pairs");
-    static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kFusedReserve;
-    static constexpr int kS8Raw = (C::kMaxSmem - kFixed - kSB * kBBytes) / kA8Bytes;
-    static constexpr int kS8 = kS8Raw < kBarSlots - kSA - kSB ? kS8Raw : kBarSlots - kSA - kSB;
-    static constexpr int kRingBytes = kSB * kBBytes + kS8 * kA8Bytes;
+    static constexpr uint32_t kTxBytes = kABytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kSmemBytes = kFixed + kRingBytes;
     static constexpr int kPf = 2;  // pair stages the producer prefetches into L2 ahead
-    // 640 threads: the roles of the bf16 kernel's warps 0..15, except that warps
-    // 4..7 convert the first box of each stage and the extra warps 16..19 the
-    // second (warp % 4 = the TMEM lane quarter, i.e. the 32 weight rows, it
-    // writes); warp 3 is idle
-    static constexpr int kThreads = 640;
-    static constexpr int kConv0 = 4, kConvExtra0 = 16, kConvWarps = 8;
-    // barrier slots in Aux's full/empty arrays
-    static constexpr int kBar8 = 0, kBarA = kS8, kBarB = kS8 + kSA;
-    static constexpr int kEmptyB = kSA == kSB ? kBarA : kBarB;  // the B ring's "empty" barriers
-    static_assert(kS8 >= 3 && kS8 + kSA + kSB <= kBarSlots, "barrier slots");
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kStages >= 3 && kStages <= kBarSlots, "pipeline depth");
     static_assert(kSmemBytes <= C::kMaxSmem, "shared memory");
-    static_assert(kACol0 + kSA * kACols <= kTmemCols && kNBuf * C::kAccCols <= kACol0, "TMEM");
+    static_assert(kNBuf * kAccCols <= kTmemCols && kNBuf >= 2, "TMEM");
 };
 
-// Four E4M3 codes (byte i = element i) -> four bf16 values, two per word, lower
-// element in the lower half.  E4M3 -> f16 -> f32 -> bf16 are all exact for E4M3
-// values (3 significand bits, exponents 2^-9 .. 2^8), NaN stays NaN.
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
+// The largest |x| of one token, published once per call by one CTA for all the
+// others: `m` first, then `gen` (release).
+struct XMax {
+    unsigned long long gen;
+    uint32_t m;
+    uint32_t pad;
+};
+
+// ---- E4M3 token operand (F8).  A bf16 row v (x rows for w13, act rows for w2)
+// is multiplied by 2^s, s chosen from the row's largest magnitude so that it
+// lands in [128, 256), and written as two E4M3 terms: hi = e4m3(v 2^s) and
+// lo = e4m3(v 2^s - hi), both rounded to nearest.  A bf16 value has 8
+// significant bits and hi keeps the leading 4, so the remainder fits lo's 4
+// significant bits: hi + lo is v 2^s exactly unless lo falls below E4M3's
+// subnormal step 2^-9, which only entries under 2^-9 of the row's maximum can
+// reach (error at most 2^-10 of the scaled unit, 2^-17 of the row maximum).
+// The product of two E4M3 values is exact in fp32, so the MMA forms the bf16
+// products and the epilogue multiplies (hi + lo) accumulators by 2^-s.
+
+// s for a row whose largest |value| has fp32 bits m (a bf16 value): 7 - its
+// exponent, within [-126, 126] so that 2^s and 2^-s are normal floats; 0 for a
+// zero or non-finite row.
+__device__ __forceinline__ int row_scale_exp(uint32_t m)
 {
-    uint32_t h0, h1;
-    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
-        : "=r"(h0), "=r"(h1)
+    if (m == 0u || m >= 0x7f800000u) return 0;
+    const int e = (int)(m >> 23) - 127;
+    return min(126, max(-126, 7 - e));
+}
+__device__ __forceinline__ float pow2f(int s) { return __int_as_float((s + 127) << 23); }
+// 2^s, or NaN for a row holding inf or NaN: such a row's outputs are NaN.
+__device__ __forceinline__ float row_scale(uint32_t m)
+{
+    return m >= 0x7f800000u ? __int_as_float(0x7fc00000) : pow2f(row_scale_exp(m));
+}
+__device__ __forceinline__ float row_descale(uint32_t m) { return pow2f(-row_scale_exp(m)); }
+
+// e4m3(a) in the low byte, e4m3(b) in the high byte (round to nearest, finite).
+__device__ __forceinline__ uint32_t e4m3x2_pack(float a, float b)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
+}
+// The two E4M3 values of the low 16 bits of w (low byte first) as floats.
+__device__ __forceinline__ float2 e4m3x2_unpack(uint32_t w)
+{
+    uint32_t h;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h)
         : "r"(w));
-    const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-    const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-    const __nv_bfloat162 b0 = __floats2bfloat162_rn(f0.x, f0.y);
-    const __nv_bfloat162 b1 = __floats2bfloat162_rn(f1.x, f1.y);
-    lo = *reinterpret_cast<const uint32_t*>(&b0);
-    hi = *reinterpret_cast<const uint32_t*>(&b1);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+// Four bf16 values (two words, element 0 in the low half of w0) times sc ->
+// their E4M3 hi and lo terms, four codes per word (element 0 in the low byte).
+__device__ __forceinline__ void split4(uint32_t w0, uint32_t w1, float sc, uint32_t& hi,
+                                       uint32_t& lo)
+{
+    const float v0 = __uint_as_float(w0 << 16) * sc, v1 = __uint_as_float(w0 & 0xffff0000u) * sc;
+    const float v2 = __uint_as_float(w1 << 16) * sc, v3 = __uint_as_float(w1 & 0xffff0000u) * sc;
+    const uint32_t h01 = e4m3x2_pack(v0, v1), h23 = e4m3x2_pack(v2, v3);
+    const float2 f01 = e4m3x2_unpack(h01), f23 = e4m3x2_unpack(h23);
+    hi = h01 | (h23 << 16);
+    lo = e4m3x2_pack(v0 - f01.x, v1 - f01.y) | (e4m3x2_pack(v2 - f23.x, v3 - f23.y) << 16);
+}
+// 16 bf16 values (K order) -> 16 hi codes and 16 lo codes.
+__device__ __forceinline__ void split16(const uint4& a, const uint4& b, float sc, uint4& hi,
+                                        uint4& lo)
+{
+    split4(a.x, a.y, sc, hi.x, lo.x);
+    split4(a.z, a.w, sc, hi.y, lo.y);
+    split4(b.x, b.y, sc, hi.z, lo.z);
+    split4(b.z, b.w, sc, hi.w, lo.w);
+}
+// fp32 bits of the largest |value| among the 8 bf16 values of v, folded into m2
+// (two 16-bit lanes).
+__device__ __forceinline__ uint32_t absmax8(uint32_t m2, const uint4& v)
+{
+    m2 = __vmaxu2(m2, v.x & 0x7fff7fffu);
+    m2 = __vmaxu2(m2, v.y & 0x7fff7fffu);
+    m2 = __vmaxu2(m2, v.z & 0x7fff7fffu);
+    return __vmaxu2(m2, v.w & 0x7fff7fffu);
 }
 
 __device__ __forceinline__ void flag_error(int32_t* err, Aux* aux)
@@ -256,6 +309,27 @@ __device__ __forceinline__ bool wait_counters(const FusedArgs& a, volatile int* 
             globaltimer_ns() - t0 > 2000000000ull)
             return false;
     }
+}
+
+// F8: the largest |x| of token t published this call (fp32 bits, into m): a
+// bounded wait for its generation word (acquire), then the value.  False on a
+// timeout, a local abort or another CTA's recorded error.
+__device__ __forceinline__ bool token_xmax(const FusedArgs& a, int t, volatile int* abort,
+                                           uint32_t& m)
+{
+    const unsigned long long* g = &a.xmax[t].gen;
+    if (ld_acquire_gpu_u64(g) != a.gen) {
+        const uint64_t t0 = globaltimer_ns();
+        for (;;) {
+            __nanosleep(64);
+            if (ld_acquire_gpu_u64(g) == a.gen) break;
+            if (*abort || *reinterpret_cast<const volatile int32_t*>(a.err) == kDeviceErrorMagic ||
+                globaltimer_ns() - t0 > 2000000000ull)
+                return false;
+        }
+    }
+    m = __ldcg(&a.xmax[t].m);
+    return true;
 }
 
 // Routes the T tokens in this CTA (every thread calls; ends with a barrier).
@@ -440,24 +514,29 @@ __device__ __forceinline__ void route_tokens(const FusedArgs& a, RouteSmem* rs, 
     __syncthreads();
 }
 
-// W8: tm_w13 / tm_w2 map E4M3 codes ([128 x 128]-byte boxes, 128-byte swizzle).
-template <int NT, bool W8>
-__global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
+// F8: E4M3 weights (kind::f8f6f4 MMAs against the split E4M3 token operand);
+// tm_w13 / tm_w2 then map E4M3 codes ([128 x 128]-byte boxes, 128-byte swizzle).
+template <int NT, bool F8>
+__global__ void __launch_bounds__(kThreads, 1)
     fused_ffn_kernel(const __grid_constant__ CUtensorMap tm_w13,
                      const __grid_constant__ CUtensorMap tm_w2,
                      const __grid_constant__ CUtensorMap tm_act, const FusedArgs a)
 {
     using C = FCfg<NT>;
-    using R8 = W8Cfg<NT>;
+    using F8C = F8Cfg<NT>;
     static_assert(NT <= 64, "weight-streaming tiles");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    constexpr int kRingBytes = W8 ? R8::kRingBytes : C::kStages * C::kStageBytes;
-    constexpr int NBUF = W8 ? R8::kNBuf : C::kNBuf;  // accumulator buffers
-    constexpr int kTmemCols = W8 ? R8::kTmemCols : C::kTmemCols;
-    uint8_t* const bring = ring;                            // W8: token tiles
-    uint8_t* const ring8 = ring + R8::kSB * R8::kBBytes;    // W8: E4M3 pair stages
+    // the ring (bf16: one 64-element K tile per stage; F8: two)
+    constexpr int kStagesM = F8 ? F8C::kStages : C::kStages;
+    constexpr int kStageBytesM = F8 ? F8C::kStageBytes : C::kStageBytes;
+    constexpr int kGM = F8 ? F8C::kG : C::kG;  // gather groups and warps per group
+    constexpr int kWM = F8 ? F8C::kW : C::kW;
+    constexpr int kAccColsM = F8 ? F8C::kAccCols : C::kAccCols;  // per accumulator buffer
+    constexpr int kRingBytes = kStagesM * kStageBytesM;
+    constexpr int NBUF = F8 ? F8C::kNBuf : C::kNBuf;  // accumulator buffers
+    constexpr int kTmemCols = F8 ? F8C::kTmemCols : C::kTmemCols;
     uint8_t* staging = ring + kRingBytes;
     Aux* aux = reinterpret_cast<Aux*>(staging + C::kStagingBytes);
     ComboScratch* combo = reinterpret_cast<ComboScratch*>(aux + 1);
@@ -465,30 +544,18 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     int4* unit_tab = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(aux) + C::kAuxBytes);
     int* tab_seq = reinterpret_cast<int*>(unit_tab + 2 * kUnitTable);
     RouteSmem* rs = reinterpret_cast<RouteSmem*>(tab_seq + kUnitTable);
-    static_assert(kRouteScratchBytes <= kRingBytes &&
-                      (W8 ? R8::kThreads : kThreads) / 32 * kMaxExperts * 4 <= kStagedLogitBytes &&
-                      (W8 ? R8::kThreads : kThreads) / 32 <= 20,
+    float* cscale = reinterpret_cast<float*>(rs + 1);  // F8: [gather warps][NT] row scales
+    // the routing scratch may run on into the epilogue staging that follows the ring
+    static_assert(kRouteScratchBytes <= kRingBytes + C::kStagingBytes &&
+                      kThreads / 32 * kMaxExperts * 4 <= kStagedLogitBytes && kThreads / 32 <= 20,
                   "routing scratch");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        if constexpr (W8) {
-            for (int s = 0; s < R8::kS8; ++s) {
-                mbar_init(&aux->full[R8::kBar8 + s], 1);  // the producer's expect_tx
-                mbar_init(&aux->empty[R8::kBar8 + s], R8::kConvWarps);
-            }
-            for (int s = 0; s < R8::kSB; ++s) {
-                mbar_init(&aux->full[R8::kBarB + s], 1);   // per stage: the gather warp
-                mbar_init(&aux->empty[R8::kBarB + s], 1);  // per slot pair (first kSB / 2)
-            }
-            for (int s = 0; s < R8::kSA; ++s) {  // per slot pair (first kSA / 2 used)
-                mbar_init(&aux->full[R8::kBarA + s], R8::kConvWarps);
-                mbar_init(&aux->empty[R8::kBarA + s], 1);
-            }
-        } else {
-            for (int s = 0; s < C::kStages; ++s) {
-                mbar_init(&aux->full[s], 1 + C::kW);
+        {
+            for (int s = 0; s < kStagesM; ++s) {
+                mbar_init(&aux->full[s], 1 + kWM);
                 mbar_init(&aux->empty[s], 1);
             }
         }
@@ -529,7 +596,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             st_release_gpu_u64(a.ready, a.gen);
         }
     }
-    route_tokens(a, rs, ring);  // the ring is free until the producer's first load
+    route_tokens(a, rs, ring);  // ring and staging are free until the first load / unit
 
     const int ntiles = rs->n_tiles;
     // w13 is not split here: its epilogue writes bf16 act directly, which each w2
@@ -539,7 +606,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     // 101.4 us decode / 360.7 us skewed decode, 4 waves 98.2 / 341.8).
     const int s2w = split_count(ntiles * a.fb2, a.s2_max, a.kt2, a.min_kt_per_split, 4);
     int ktps2 = (a.kt2 + s2w - 1) / s2w;
-    if (W8) ktps2 = (ktps2 + 1) & ~1;  // whole pair stages
+    if (F8) ktps2 = (ktps2 + 1) & ~1;  // whole pair stages
     const int S2 = (a.kt2 + ktps2 - 1) / ktps2;  // every slice non-empty
     const int U13 = ntiles * a.fb13;
     const int U2 = ntiles * a.fb2 * S2;
@@ -640,13 +707,14 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t pol = l2_policy_evict_first();  // each weight block is read once
-            // W8: the E4M3 ring (its barriers are full/empty[0, kS8))
-            constexpr int NS = W8 ? R8::kS8 : C::kStages;
-            constexpr int kStBytes = W8 ? R8::kA8Bytes : C::kStageBytes;
-            constexpr int kBox1 = W8 ? kBM * 2 * kBK : kATileBytes;  // offset of the second box
-            constexpr int kKtStep = W8 ? 2 : 1;  // K tiles per ring stage
-            constexpr uint32_t kTx = W8 ? (uint32_t)R8::kA8Bytes : C::kTxBytes;
-            uint8_t* const pring = W8 ? ring8 : ring;
+            // F8: the single ring, two E4M3 boxes per stage
+            constexpr int NS = kStagesM;
+            constexpr int kStBytes = kStageBytesM;
+            constexpr int kBox1 = F8 ? kBM * 2 * kBK : kATileBytes;  // second box
+            constexpr int kKtStep = F8 ? 2 : 1;  // K tiles per ring stage
+            constexpr uint32_t kTx = F8 ? F8C::kTxBytes : C::kTxBytes;
+            constexpr int kPf = F8C::kPf;
+            uint8_t* const pring = ring;
             int stage = 0;
             uint32_t phase = 0;
             int fills = 0;  // ring stage fills so far (fill q went to stage q % stages)
@@ -682,11 +750,11 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 const int row0 = un.ph ? t.expert * a.H + un.fb * 2 * kBM
                                        : t.expert * 2 * a.I + un.fb * kBM;
                 const int row1 = un.ph ? row0 + kBM : row0 + a.I;
-                if constexpr (W8) {
+                if constexpr (F8) {
                     // the E4M3 ring holds fewer K tiles than the bf16 one: pair
                     // stages kPf ahead of the TMA go to L2 now, to keep more weight
                     // bytes in flight
-                    for (int kt = un.kt0 + 2; kt < min(un.kt1, un.kt0 + 2 * R8::kPf); kt += 2) {
+                    for (int kt = un.kt0 + 2; kt < min(un.kt1, un.kt0 + 2 * kPf); kt += 2) {
                         tma_prefetch_l2_2d(tm, kt * kBK, row0);
                         tma_prefetch_l2_2d(tm, kt * kBK, row1);
                     }
@@ -701,9 +769,9 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                     mbar_arrive_expect_tx(&aux->full[stage], kTx);
                     tma_load_2d(st, tm, &aux->full[stage], kt * kBK, row0, pol);
                     tma_load_2d(st + kBox1, tm, &aux->full[stage], kt * kBK, row1, pol);
-                    if (W8 && kt + 2 * R8::kPf < un.kt1) {
-                        tma_prefetch_l2_2d(tm, (kt + 2 * R8::kPf) * kBK, row0);
-                        tma_prefetch_l2_2d(tm, (kt + 2 * R8::kPf) * kBK, row1);
+                    if (F8 && kt + 2 * kPf < un.kt1) {
+                        tma_prefetch_l2_2d(tm, (kt + 2 * kPf) * kBK, row0);
+                        tma_prefetch_l2_2d(tm, (kt + 2 * kPf) * kBK, row1);
                     }
                     ++fills;
                     if (++stage == NS) {
@@ -729,7 +797,6 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int q = 0;  // W8: global stage number
             bool ok = true;
             for (int lu = 0; ok; ++lu) {
                 const Unit un = get(lu);
@@ -743,64 +810,46 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 }
                 tc_fence_after();
                 const int n = (t.rows + 15) & ~15;
-                const uint32_t idesc = umma_idesc_bf16(kBM, n);
-                const uint32_t d0 = tmem_base + (uint32_t)(b * C::kAccCols);
-                for (int kt = un.kt0; kt < un.kt1; ++kt) {
+                // F8: hi and lo terms of the n token rows make the MMA's 2 n columns
+                const uint32_t idesc = F8 ? umma_idesc_e4m3(kBM, 2 * n) : umma_idesc_bf16(kBM, n);
+                const uint32_t d0 = tmem_base + (uint32_t)(b * kAccColsM);
+                for (int kt = un.kt0; kt < un.kt1; kt += (F8 ? 2 : 1)) {
                     uint32_t st, bt;
-                    if constexpr (W8) {
-                        // A arrives a pair of K tiles at a time (slots 2 pa, 2 pa + 1)
-                        const int sa = q % R8::kSA, sb = q % R8::kSB;
-                        const int pa = (q >> 1) % (R8::kSA / 2);
-                        if (((q & 1) == 0 &&
-                             !mbar_wait(&aux->full[R8::kBarA + pa],
-                                        (uint32_t)(((q >> 1) / (R8::kSA / 2)) & 1), abort_flag)) ||
-                            !mbar_wait(&aux->full[R8::kBarB + sb], (uint32_t)((q / R8::kSB) & 1),
-                                       abort_flag)) {
-                            flag_error(a.err, aux);
-                            ok = false;
-                            break;
-                        }
-                        // the x rows of B were written by cp.async (generic proxy)
-                        fence_proxy_async_smem();
-                        st = tmem_base + R8::kACol0 + sa * R8::kACols;  // A in TMEM
-                        bt = smem_u32(bring + sb * R8::kBBytes);
-                    } else {
+                    {
                         if (!mbar_wait(&aux->full[stage], phase, abort_flag)) {
                             flag_error(a.err, aux);
                             ok = false;
                             break;
                         }
-                        st = smem_u32(ring + stage * C::kStageBytes);
-                        bt = st + C::kNA * kATileBytes;
+                        st = smem_u32(ring + stage * kStageBytesM);
+                        bt = st + (F8 ? F8C::kABytes : C::kNA * kATileBytes);
                     }
                     tc_fence_after();
+                    if constexpr (F8) {
+                        // 128 K codes per stage, 32 per MMA: both boxes against the
+                        // same token operand
 #pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        const uint32_t acc = (kt > un.kt0 || kk > 0) ? 1u : 0u;
-                        const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
-                        if constexpr (W8) {  // K step kk: 8 columns of each converted tile
-                            umma_bf16_ts(d0, st + kk * (kUmmaK / 2), bdesc, idesc, acc);
-                            umma_bf16_ts(d0 + NT, st + R8::kACols / 2 + kk * (kUmmaK / 2), bdesc,
-                                         idesc, acc);
-                        } else {
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (kt > un.kt0 || kk > 0) ? 1u : 0u;
+                            const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
+                            umma_e4m3(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
+                            umma_e4m3(d0 + 2 * NT, umma_desc_sw128(st + F8C::kBoxBytes + kk * 32),
+                                      bdesc, idesc, acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                            const uint32_t acc = (kt > un.kt0 || kk > 0) ? 1u : 0u;
+                            const uint64_t bdesc = umma_desc_sw128(bt + kk * 32);
                             umma_bf16(d0, umma_desc_sw128(st + kk * 32), bdesc, idesc, acc);
                             umma_bf16(d0 + NT, umma_desc_sw128(st + kATileBytes + kk * 32), bdesc,
                                       idesc, acc);
                         }
                     }
-                    if constexpr (W8) {  // free the A and B slot pairs when read
-                        if (q & 1) {
-                            umma_commit(&aux->empty[R8::kBarA + (q >> 1) % (R8::kSA / 2)]);
-                            if constexpr (R8::kSA != R8::kSB)
-                                umma_commit(&aux->empty[R8::kBarB + (q >> 1) % (R8::kSB / 2)]);
-                        }
-                        ++q;
-                    } else {
-                        umma_commit(&aux->empty[stage]);  // frees the smem stage when read
-                        if (++stage == C::kStages) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
+                    umma_commit(&aux->empty[stage]);  // frees the smem stage when read
+                    if (++stage == kStagesM) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
                 if (ok) umma_commit(&aux->tfull[b]);
@@ -810,146 +859,119 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             volatile int never = 0;
             if (!mbar_wait(&aux->drain, 0, &never, 500000000ull)) atomicExch(a.err, kDeviceErrorMagic);
         }
-    } else if (W8 && warp == 2) {
-        // ------------------------------------------------------------ token operand (W8)
-        // One warp fills the B ring: x rows by cp.async, each lane's copies arriving
-        // on the stage's barrier when they land, or one act TMA.  Nothing here waits
-        // for its own copies, so the ring runs kSB stages ahead of the MMA.
-        int* my_off = tok_off;
-        const uint64_t keep = l2_policy_evict_last();  // x / act rows are re-read per block
-        int q = 0;
-        int cur_tile = -1, cur_ph = -1, ready_tile = -1;
-        int last_tma[R8::kSB];  // stage of each slot's latest use when that was a TMA, else -1
-        for (int sb = 0; sb < R8::kSB; ++sb) last_tma[sb] = -1;
-        bool ok = true;
-        bool counters = false;
-        for (int i = 0; ok; ++i) {
-            const Unit un = get(i);
-            if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
-            const Unit& t = un;
-            if (un.ph == 1 && un.tile != ready_tile) {
-                // every w13 unit of this tile has stored its act rows
-                if ((!counters &&
-                     !(counters = __all_sync(0xffffffffu, wait_counters(a, abort_flag)))) ||
-                    !warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
-                    if (lane == 0) flag_error(a.err, aux);
-                    ok = false;
-                    break;
-                }
-                fence_proxy_async_global();  // the act TMA reads after the acquire
-                ready_tile = un.tile;
-            }
-            if (un.tile != cur_tile || un.ph != cur_ph) {
-                __syncwarp();  // earlier copies' addresses are all issued
-                if (un.ph == 0)
-                    for (int j = lane; j < t.rows; j += 32)
-                        my_off[j] = (rs->rows[t.row_start + j] / a.k) * a.H;
-                __syncwarp();
-                cur_tile = un.tile;
-                cur_ph = un.ph;
-            }
-            for (int kt = un.kt0; kt < un.kt1; ++kt, ++q) {
-                const int sb = q % R8::kSB, pb = (q >> 1) % (R8::kSB / 2);
-                uint64_t* fb = &aux->full[R8::kBarB + sb];
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(&aux->empty[R8::kEmptyB + pb],
-                                          (uint32_t)((((q >> 1) / (R8::kSB / 2)) & 1) ^ 1),
-                                          abort_flag))) {
-                    if (lane == 0) flag_error(a.err, aux);
-                    ok = false;
-                    break;
-                }
-                uint8_t* btile = bring + sb * R8::kBBytes;
-                if (un.ph == 1) {
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(fb, R8::kBBytes);
-                        tma_load_2d_nohint(btile, &tm_act, fb, 0, kt * a.R + t.row_start);
-                    }
-                    last_tma[sb] = q;
-                    continue;
-                }
-                last_tma[sb] = -1;
-                const uint32_t bt = smem_u32(btile);
-                const __nv_bfloat16* src0 = a.x + kt * kBK;
-                for (int c8 = lane; c8 < t.rows * 8; c8 += 32) {
-                    const int j = c8 >> 3, c = c8 & 7;
-                    cp_async_16_hint(bt + j * 128 + ((c ^ (j & 7)) << 4), src0 + my_off[j] + c * 8,
-                                     keep);
-                }
-                cp_async_mbar_arrive(fb);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(fb);
-            }
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        if (lane == 0 && (!ok || *abort_flag)) {
-            // act TMAs still in flight land before the CTA can exit
-            for (int sb = 0; sb < R8::kSB; ++sb)
-                if (last_tma[sb] >= 0) {
-                    volatile int never = 0;
-                    mbar_wait(&aux->full[R8::kBarB + sb], (uint32_t)((last_tma[sb] / R8::kSB) & 1),
-                              &never, 500000000ull);
-                }
-        }
-    } else if (W8 && ((warp >= R8::kConv0 && warp < kEpiWarp0) || warp >= R8::kConvExtra0)) {
-        // ------------------------------------------------------------ converters (W8)
-        // Thread = weight row r = 32 (warp % 4) + lane of box `box` (gate / up, or
-        // the two w2 row blocks).  Per pair stage, for each of its two K tiles, it
-        // reads its row's 64 codes (four 16-byte chunks; in the 128-byte swizzle, 8
-        // consecutive rows put a chunk in 8 distinct bank groups, so the loads do
-        // not conflict), widens them to 32 bf16 pairs and stores them to 32 TMEM
-        // columns of lane r; then one arrival hands both K tiles to the MMA.
-        const int qd = warp & 3;
-        const int box = warp >= R8::kConvExtra0 ? 1 : 0;
-        const int r = qd * 32 + lane;
-        const uint32_t tst = tmem_base + ((uint32_t)(qd * 32) << 16) + R8::kACol0 +
-                             box * (R8::kACols / 2);
-        int q = 0;
-        bool ok = true;
-        for (int i = 0; ok; ++i) {
-            const Unit un = get(i);
-            if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
-            for (int kt = un.kt0; kt < un.kt1; kt += 2, q += 2) {  // one pair stage
-                const int pq = q >> 1, s8 = pq % R8::kS8, pa = pq % (R8::kSA / 2);
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(&aux->empty[R8::kBarA + pa],
-                                          (uint32_t)(((pq / (R8::kSA / 2)) & 1) ^ 1), abort_flag)) ||
-                    !__all_sync(0xffffffffu, mbar_wait(&aux->full[R8::kBar8 + s8],
-                                                       (uint32_t)((pq / R8::kS8) & 1), abort_flag))) {
-                    if (lane == 0) flag_error(a.err, aux);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();  // the MMA that read these columns has completed
-                const uint8_t* src = ring8 + s8 * R8::kA8Bytes + box * R8::kBoxBytes + r * 128;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {  // K tile kt + h: A slot 2 pa + h
-                    uint32_t o[32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {  // K elements 16 c .. 16 c + 15 of the tile
-                        const uint4 v =
-                            *reinterpret_cast<const uint4*>(src + (((c + 4 * h) ^ (r & 7)) << 4));
-                        e4m3x4_to_bf16x4(v.x, o[8 * c + 0], o[8 * c + 1]);
-                        e4m3x4_to_bf16x4(v.y, o[8 * c + 2], o[8 * c + 3]);
-                        e4m3x4_to_bf16x4(v.z, o[8 * c + 4], o[8 * c + 5]);
-                        e4m3x4_to_bf16x4(v.w, o[8 * c + 6], o[8 * c + 7]);
-                    }
-                    tmem_st32(tst + (2 * pa + h) * R8::kACols, o);
-                }
-                tmem_st_wait();  // both K tiles' stores
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&aux->full[R8::kBarA + pa]);
-                    mbar_arrive(&aux->empty[R8::kBar8 + s8]);  // pair stage read
-                }
-            }
-        }
     } else if (warp < 2 + kGatherWarps) {
         // ------------------------------------------------------------ gather
-        // (W8: only warp 3 gets here, and it has nothing to do)
-        if (!W8 && warp - 2 < C::kG * C::kW) {
+        if (F8 && warp - 2 < kGM * kWM) {
+            // F8: the E4M3 token operand.  Group g (W warps) fills stages g, g + G,
+            // ... of the ring: per stage, each row's 128 bf16 values (x for w13,
+            // act for w2) scaled by its row's 2^s and split into hi and lo codes,
+            // stored into the stage's B rows j and n + j (128-byte swizzle); then
+            // a proxy fence and one arrival per warp.
+            constexpr int G = kGM, W = kWM;
+            const int g = (warp - 2) / W, wi = (warp - 2) % W;
+            int* my_off = tok_off + (warp - 2) * NT;   // w13: element offset of each x row
+            float* my_sc = cscale + (warp - 2) * NT;   // 2^s of each row
+            int q = 0;  // global stage sequence number (same as the producer's)
+            int cur_tile = -1, cur_ph = -1, ready_tile = -1;
+            bool ok = true;
+            bool counters = false;
+            for (int i = 0; ok; ++i) {
+                const Unit un = get(i);
+                if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
+                const int nst = (un.kt1 - un.kt0) >> 1;  // pair stages of the unit
+                int sidx = ((g - q % G) + G) % G;       // first one this group owns
+                const int q_unit0 = q;
+                q += nst;
+                if (sidx >= nst) continue;
+                const Unit& t = un;
+                if (un.ph == 1 && un.tile != ready_tile) {
+                    // every w13 unit of this tile has stored its act rows and maxima
+                    if ((!counters &&
+                         !(counters = __all_sync(0xffffffffu, wait_counters(a, abort_flag)))) ||
+                        !warp_wait_count(a.tile_ready + un.tile, tile_target, abort_flag, a.err)) {
+                        if (lane == 0) flag_error(a.err, aux);
+                        ok = false;
+                        break;
+                    }
+                    ready_tile = un.tile;
+                }
+                if (un.tile != cur_tile || un.ph != cur_ph) {
+                    __syncwarp();  // the previous tile's rows are all converted
+                    bool got = true;
+                    for (int j = lane; j < t.rows; j += 32) {
+                        uint32_t m = 0;
+                        if (un.ph == 0) {
+                            const int tok = rs->rows[t.row_start + j] / a.k;
+                            my_off[j] = tok * a.H;
+                            got = token_xmax(a, tok, abort_flag, m) && got;
+                        } else {
+                            m = (uint32_t)ld_acquire_gpu(
+                                reinterpret_cast<const int*>(a.act_max) + t.row_start + j);
+                        }
+                        my_sc[j] = row_scale(m);
+                    }
+                    if (__any_sync(0xffffffffu, !got)) {
+                        if (lane == 0) flag_error(a.err, aux);
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    cur_tile = un.tile;
+                    cur_ph = un.ph;
+                }
+                const int n = (t.rows + 15) & ~15;
+                const int ntask = t.rows * 8;  // (row, 16-element chunk) pairs
+                for (; sidx < nst; sidx += G) {
+                    const int qq = q_unit0 + sidx;
+                    const int stage = qq % kStagesM;
+                    const uint32_t phase = (uint32_t)((qq / kStagesM) & 1);
+                    if (!__all_sync(0xffffffffu, mbar_wait(&aux->empty[stage], phase ^ 1u,
+                                                           abort_flag))) {
+                        if (lane == 0) flag_error(a.err, aux);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* btile = ring + stage * kStageBytesM + F8C::kABytes;
+                    const int kt = un.kt0 + 2 * sidx;  // the stage's first K tile
+                    // four tasks per lane in flight: loads first, then the splits
+                    for (int base = lane + 32 * wi; base < ntask; base += 4 * 32 * W) {
+                        uint4 v[4][2];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int c8 = base + u * 32 * W;
+                            if (c8 < ntask) {
+                                const int j = c8 >> 3, c = c8 & 7;
+                                const uint4* src =
+                                    un.ph == 0
+                                        ? reinterpret_cast<const uint4*>(a.x + my_off[j] + kt * kBK +
+                                                                         c * 16)
+                                        // act, K-blocked: block kt + c / 4, elements (c % 4) * 16 ..
+                                        : reinterpret_cast<const uint4*>(
+                                              a.act + ((size_t)(kt + (c >> 2)) * a.R + t.row_start + j) *
+                                                          kBK +
+                                              (c & 3) * 16);
+                                v[u][0] = __ldcg(src);
+                                v[u][1] = __ldcg(src + 1);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int c8 = base + u * 32 * W;
+                            if (c8 < ntask) {
+                                const int j = c8 >> 3, c = c8 & 7, jl = n + j;
+                                uint4 hi, lo;
+                                split16(v[u][0], v[u][1], my_sc[j], hi, lo);
+                                *reinterpret_cast<uint4*>(btile + j * 128 + ((c ^ (j & 7)) << 4)) = hi;
+                                *reinterpret_cast<uint4*>(btile + jl * 128 + ((c ^ (jl & 7)) << 4)) = lo;
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();  // generic stores, read by the MMA
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aux->full[stage]);
+                }
+            }
+        } else if (!F8 && warp - 2 < C::kG * C::kW) {
             constexpr int G = C::kG, W = C::kW;
             const int g = (warp - 2) / W, wi = (warp - 2) % W;
             int* my_off = tok_off + (warp - 2) * NT;
@@ -1040,6 +1062,29 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
         const int f_local = qw * 32 + lane;       // feature inside the 128-row block
         uint8_t* gstage = staging + grp * 2 * (kStageRows * kStageRowBytes);
         int chunk = 0;  // staging chunks issued by this group (buffer parity)
+        if constexpr (F8) {
+            // publish the largest |x| of tokens b, b + G, ... for every CTA's token
+            // operand (first thing, so no CTA waits long for it): all eight warps
+            // read the row, reduce, and one thread writes the value, then the
+            // call's generation with release
+            const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..255
+            uint32_t* red = reinterpret_cast<uint32_t*>(staging);
+            for (int tk = blockIdx.x; tk < a.T; tk += gridDim.x) {
+                const uint4* row = reinterpret_cast<const uint4*>(a.x + (size_t)tk * a.H);
+                uint32_t m2 = 0;
+                for (int i = et; i < a.H / 8; i += 256) m2 = absmax8(m2, __ldcg(row + i));
+                const uint32_t m = __reduce_max_sync(0xffffffffu, max(m2 & 0xffffu, m2 >> 16) << 16);
+                if (lane == 0) red[warp - kEpiWarp0] = m;
+                named_bar_sync(3, 256);
+                if (et == 0) {
+                    uint32_t mm = 0;
+                    for (int w = 0; w < 8; ++w) mm = max(mm, red[w]);
+                    a.xmax[tk].m = mm;
+                    st_release_gpu_u64(&a.xmax[tk].gen, a.gen);
+                }
+                named_bar_sync(3, 256);  // red is rewritten for the next token
+            }
+        }
         // every epilogue thread publishes to (or waits on) the counters: before its
         // first unit's accumulator is even ready, CTA 0 has long zeroed them (the
         // outcome is made the same in all four warps of the group)
@@ -1050,10 +1095,10 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             const Unit& t = un;
             const int b = lu % NBUF;
             const uint32_t aphase = (uint32_t)((lu / NBUF) & 1);
-            // W8: this thread's two weight-row scales (gate and up rows, or output
+            // F8: this thread's two weight-row scales (gate and up rows, or output
             // features f and f + 128), loaded before the accumulator wait
             float sc0 = 1.f, sc1 = 1.f;
-            if constexpr (W8) {
+            if constexpr (F8) {
                 if (un.ph == 0) {
                     const float* sp = a.s13 + (size_t)un.expert * 2 * a.I + un.fb * kBM + f_local;
                     sc0 = __ldg(sp);
@@ -1065,6 +1110,27 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                     if (f2 + kBM < a.H) sc1 = __ldg(sp + kBM);
                 }
             }
+            // F8: 2^-s of the token column jbeg + lane of this group, each lane
+            // loading one column's maximum (all at once; the chunks below take
+            // theirs by shuffle).  w13: the tokens' published x maxima, fetched
+            // while the MMAs run; w2: the act maxima, complete once this unit's
+            // operand was built, so fetched after the accumulator wait.
+            float my_ds = 1.f;
+            auto load_ds = [&](int ph_) {
+                const int j = grp * (NT / 2) + lane;
+                uint32_t m = 0;
+                if (j < min(t.rows, (grp + 1) * (NT / 2))) {
+                    if (ph_ == 0) {
+                        if (!token_xmax(a, rs->rows[t.row_start + j] / a.k, abort_flag, m))
+                            flag_error(a.err, aux);
+                    } else {
+                        m = (uint32_t)ld_acquire_gpu(reinterpret_cast<const int*>(a.act_max) +
+                                                     t.row_start + j);
+                    }
+                }
+                my_ds = row_descale(m);
+            };
+            if (F8 && un.ph == 0) load_ds(0);
             bool got = false;
             if (un.ph < kUnitEnd) {
                 got = mbar_wait(&aux->tfull[b], aphase, abort_flag);
@@ -1079,8 +1145,16 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
             // (accumulator 1); w2: output features f and f + 128
             const int f = (ph == 0 ? un.fb * kBM : un.fb * 2 * kBM) + f_local;
             const bool f1_ok = ph == 0 || f + kBM < a.H;
-            const uint32_t tacc = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)(b * C::kAccCols);
+            const uint32_t tacc = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)(b * kAccColsM);
             const int jbeg = grp * (NT / 2), jend = min(t.rows, (grp + 1) * (NT / 2));
+            // F8: the lo terms' columns start at n; the second box's at 2 NT
+            const int n8 = (t.rows + 15) & ~15;
+            constexpr uint32_t kBox1Col = F8 ? 2 * NT : NT;
+            if (F8 && ph == 1) load_ds(1);
+            // 2^-s of column j of the group (lanes hold them; all lanes call)
+            auto col_descale = [&](int j) -> float {
+                return __shfl_sync(0xffffffffu, my_ds, (j - jbeg) & 31);
+            };
             if (jbeg >= jend) {  // this group had no columns of the unit
                 tc_fence_before();
                 __syncwarp();
@@ -1093,15 +1167,27 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 const int vec_per_row = row_bytes / 16;
                 for (int j0 = jbeg; j0 < jend; j0 += kStageRows) {
                     uint32_t gv[8], vv[8];
-                    tmem_ld8(tacc + j0, gv);
-                    tmem_ld8(tacc + NT + j0, vv);
-                    tmem_ld_wait();
-                    if constexpr (W8) {
+                    if constexpr (F8) {
+                        uint32_t gl[8], vl[8];
+                        float ds[kStageRows];
+#pragma unroll
+                        for (int jj = 0; jj < kStageRows; ++jj) ds[jj] = col_descale(j0 + jj);
+                        tmem_ld8(tacc + j0, gv);
+                        tmem_ld8(tacc + n8 + j0, gl);
+                        tmem_ld8(tacc + kBox1Col + j0, vv);
+                        tmem_ld8(tacc + kBox1Col + n8 + j0, vl);
+                        tmem_ld_wait();
 #pragma unroll
                         for (int jj = 0; jj < kStageRows; ++jj) {
-                            gv[jj] = __float_as_uint(__uint_as_float(gv[jj]) * sc0);
-                            vv[jj] = __float_as_uint(__uint_as_float(vv[jj]) * sc1);
+                            const float g = __uint_as_float(gv[jj]) + __uint_as_float(gl[jj]);
+                            const float u = __uint_as_float(vv[jj]) + __uint_as_float(vl[jj]);
+                            gv[jj] = __float_as_uint(g * ds[jj] * sc0);
+                            vv[jj] = __float_as_uint(u * ds[jj] * sc1);
                         }
+                    } else {
+                        tmem_ld8(tacc + j0, gv);
+                        tmem_ld8(tacc + NT + j0, vv);
+                        tmem_ld_wait();
                     }
                     if (j0 + kStageRows >= jend) {  // accumulator drained: let the MMA go on
                         tc_fence_before();
@@ -1113,8 +1199,15 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                     for (int jj = 0; jj < kStageRows; ++jj) {
                         __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(buf + jj * kStageRowBytes);
                         if (ph == 0) {
-                            row[f_local] = __float2bfloat16_rn(
+                            const __nv_bfloat16 av = __float2bfloat16_rn(
                                 silu_mul(__uint_as_float(gv[jj]), __uint_as_float(vv[jj])));
+                            row[f_local] = av;
+                            if constexpr (F8) {  // the row's largest |act|, for w2's operand
+                                const uint32_t m = __reduce_max_sync(
+                                    0xffffffffu, ((uint32_t)__bfloat16_as_ushort(av) & 0x7fffu) << 16);
+                                if (lane == 0 && j0 + jj < jend)
+                                    atomicMax(a.act_max + t.row_start + j0 + jj, m);
+                            }
                         } else {
                             row[f_local] = __float2bfloat16_rn(__uint_as_float(gv[jj]));
                             row[kBM + f_local] = __float2bfloat16_rn(__uint_as_float(vv[jj]));
@@ -1138,9 +1231,24 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                 constexpr int kCols = kEpiCols<NT>;
                 for (int j0 = jbeg; j0 < jend; j0 += kCols) {
                     uint32_t gv[kCols], vv[kCols];
-                    tmem_ld_cols(tacc + j0, gv);
-                    tmem_ld_cols(tacc + NT + j0, vv);
-                    tmem_ld_wait();
+                    if constexpr (F8) {
+                        uint32_t gl[kCols], vl[kCols];
+                        tmem_ld_cols(tacc + j0, gv);
+                        tmem_ld_cols(tacc + n8 + j0, gl);
+                        tmem_ld_cols(tacc + kBox1Col + j0, vv);
+                        tmem_ld_cols(tacc + kBox1Col + n8 + j0, vl);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int jj = 0; jj < kCols; ++jj) {
+                            const float ds = col_descale(j0 + jj);
+                            gv[jj] = __float_as_uint((__uint_as_float(gv[jj]) + __uint_as_float(gl[jj])) * ds);
+                            vv[jj] = __float_as_uint((__uint_as_float(vv[jj]) + __uint_as_float(vl[jj])) * ds);
+                        }
+                    } else {
+                        tmem_ld_cols(tacc + j0, gv);
+                        tmem_ld_cols(tacc + NT + j0, vv);
+                        tmem_ld_wait();
+                    }
 #pragma unroll
                     for (int jj = 0; jj < kCols; ++jj) {
                         const int j = j0 + jj;
@@ -1150,7 +1258,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
                             const int r = rs->rows[p];
                             float* prow = a.part2 + ((size_t)un.split * a.R + r) * a.H;
                             float g0 = __uint_as_float(gv[jj]), g1 = __uint_as_float(vv[jj]);
-                            if constexpr (W8) {
+                            if constexpr (F8) {
                                 g0 *= sc0;
                                 g1 *= sc1;
                             }
@@ -1250,7 +1358,7 @@ __global__ void __launch_bounds__(W8 ? W8Cfg<NT>::kThreads : kThreads, 1)
     }
 }
 
-template <int NT, bool W8>
+template <int NT, bool F8>
 cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const CUtensorMap& ta,
                             const FusedArgs& a, int grid, cudaStream_t st)
 {
@@ -1259,13 +1367,12 @@ cudaError_t launch_fused_nt(const CUtensorMap& t13, const CUtensorMap& t2, const
     // table and the routing tables follow the aux area
     static_assert(sizeof(Aux) + sizeof(ComboScratch) <= 1024, "aux area");
     static_assert(C::kAuxBytes % 16 == 0 && kUnitTableBytes % 16 == 0, "table alignment");
-    constexpr int smem = W8 ? W8Cfg<NT>::kSmemBytes : C::kSmemBytes + kFusedReserve;
+    constexpr int smem = F8 ? F8Cfg<NT>::kSmemBytes : C::kSmemBytes + kFusedReserve;
     static_assert(smem <= C::kMaxSmem, "shared memory");
-    auto kern = fused_ffn_kernel<NT, W8>;
+    auto kern = fused_ffn_kernel<NT, F8>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    return launch_pdl(kern, dim3(grid), dim3(W8 ? W8Cfg<NT>::kThreads : kThreads), smem, st, t13,
-                      t2, ta, a);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, t13, t2, ta, a);
 }
 
 }  // namespace
@@ -1279,9 +1386,10 @@ bool fused_ffn_eligible(int T, int E, int k, int H, int I, const FfnPlan& plan)
            E <= kMaxExperts && plan.s2_max <= kMaxSplits;
 }
 
-int fused_ffn_counters(int T, int H, const FfnPlan& plan)
+int fused_ffn_counters(int T, int k, int H, const FfnPlan& plan)
 {
-    return plan.max_tiles + T * ((H / kBM + 1) / 2) + 1;
+    // tile_ready, token_ready, w2_next, then (E4M3 weights) act_max
+    return plan.max_tiles + T * ((H / kBM + 1) / 2) + 1 + T * k;
 }
 
 cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, int I,
@@ -1314,7 +1422,9 @@ cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, 
     a.tile_ready = b.counters;
     a.token_ready = b.counters + plan.max_tiles;
     a.w2_next = a.token_ready + (size_t)T * ((H / kBM + 1) / 2);
-    a.n_counters = fused_ffn_counters(T, H, plan);
+    a.act_max = reinterpret_cast<uint32_t*>(a.w2_next + 1);
+    a.n_counters = fused_ffn_counters(T, k, H, plan);
+    a.xmax = static_cast<XMax*>(b.xmax);
     a.ready = b.ready;
     a.gen = b.gen;
     a.split_out = b.splits;

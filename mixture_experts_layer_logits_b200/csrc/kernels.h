@@ -192,12 +192,13 @@ struct FusedBuffers {
     void* out;         // bf16 [T, H]
     int32_t* counters; // [fused_ffn_counters()]
     unsigned long long* ready;
+    void* xmax;        // [T] 16-byte words (largest |x| per token, E4M3 weights)
     unsigned long long gen;
     int32_t* splits;   // [2]
     int32_t* err;
 };
 bool fused_ffn_eligible(int T, int E, int k, int H, int I, const FfnPlan& plan);
-int fused_ffn_counters(int T, int H, const FfnPlan& plan);
+int fused_ffn_counters(int T, int k, int H, const FfnPlan& plan);
 cudaError_t launch_fused_ffn(const FusedBuffers& b, int T, int E, int k, int H, int I,
                              const FfnPlan& plan, cudaStream_t st);
 // moe_forward uses the fused launch where eligible unless MOE_DISABLE_FUSED=1.

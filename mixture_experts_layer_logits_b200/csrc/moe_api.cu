@@ -80,7 +80,7 @@ bool combine_shape_ok(const moe_shape_t& s)
 
 struct Layout {
     size_t err, ids, weights, offsets, rows, tiles, num_tiles, splits, chunks, bar, partials, act,
-        y, partials2, counters, ready, total;
+        y, partials2, counters, ready, xmax, total;
     int max_chunks;  // chunk rows of the multi-CTA permutation's count table
     FfnPlan plan;
     bool ffn;
@@ -125,9 +125,10 @@ Layout layout_for(const moe_shape_t& s)
         L.fused = fused_ffn_eligible(s.T, s.E, s.top_k, H, I, L.plan);
         if (L.fused) {
             L.partials2 = take(p2 * sizeof(float));
-            L.n_counters = fused_ffn_counters(s.T, H, L.plan);
+            L.n_counters = fused_ffn_counters(s.T, s.top_k, H, L.plan);
             L.counters = take((size_t)L.n_counters * sizeof(int32_t));
             L.ready = take(sizeof(unsigned long long));
+            L.xmax = take((size_t)s.T * 16);
         }
     }
     L.total = off;
@@ -364,6 +365,7 @@ static moe_status_t forward_impl(const moe_bf16_t* x, const float* logits, const
         b.out = out;
         b.counters = at<int32_t>(ws, L.counters);
         b.ready = at<unsigned long long>(ws, L.ready);
+        b.xmax = at<void>(ws, L.xmax);
         b.gen = next_generation();
         b.splits = at<int32_t>(ws, L.splits);
         b.err = at<int32_t>(ws, L.err);

@@ -152,3 +152,35 @@ def test_forward_w8_rejects_bf16_weights_and_wrong_scales():
     with pytest.raises(ValueError):
         moe.moe_forward_w8(d["x"], d["logits"], d["q13"], d["s13"][:, :-1], d["q2"], d["s2"],
                            w.k)
+
+
+def test_forward_w8_rows_of_different_magnitudes():
+    """Token rows scaled by powers of two from 2^-40 to 2^40, one row all zero and
+    one holding a few large entries among tiny ones: each token's output is
+    checked against the oracle on its own scale (the layer is linear in each
+    x row up to SwiGLU, so a wrong per-row operand scale shows in that row)."""
+    w = wl.custom("row_scales", 16, 16, 4, 512, 256)
+    d = w8_inputs(w, seed=11)
+    x = d["x"].float()
+    exps = [-40, -30, -24, -12, -6, -1, 0, 1, 3, 7, 12, 20, 30, 40, 0, 0]
+    for t, e in enumerate(exps):
+        x[t] *= 2.0 ** e
+    x[14] = 0.0
+    x[15] *= 2.0 ** -30
+    x[15, ::97] = 3.0  # a handful of entries 2^30 above the rest
+    d["x"] = x.to(torch.bfloat16)
+    out, ids, wts, off, rows = run_w8(w, d)
+    ref = oracle.forward_w8(host_bits(d["x"]), host_f32(d["logits"]), host_u8(d["q13"]),
+                            host_f32(d["s13"]), host_u8(d["q2"]), host_f32(d["s2"]), w.k)
+    assert_routing_equal(ids, wts, ref["topk_ids"], ref["topk_weights"])
+    got = out.float().cpu().double().numpy()
+    assert np.all(got[14] == 0.0)
+    for t in range(w.T):
+        if t == 14:
+            continue
+        r = ref["out"][t]
+        scale = np.abs(r).max()
+        assert scale > 0 and np.isfinite(scale), t
+        err = np.abs(got[t] - r).max()
+        assert err <= 2e-2 * scale, f"token {t}: max|err| {err:.3e} vs max|ref| {scale:.3e}"
+        assert np.abs(got[t] - r).sum() <= 5e-3 * np.abs(r).sum(), f"token {t}: mean error"
