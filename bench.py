@@ -54,12 +54,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (workload, kernel).  An entry is removed when its kernel changes, until it is
 # captured again.
 NCU_TRAFFIC = {
-    ("prefill", "w13"): 3_695_239_424 + 205_527_296,
-    ("prefill", "w2"): 1_815_046_656 + 509_628_928,
-    ("decode", "fused_ffn"): 509_756_416 + 3_208_192,
-    ("decode+e4m3", "fused_ffn"): 256_564_480 + 3_503_616,
-    ("skewed_decode+e4m3", "fused_ffn"): 1_074_733_312 + 8_154_112,
-    ("routing_stress", "route"): 67_145_728 + 139_776,
+    ("prefill", "w13"): 3_711_779_328 + 205_911_296,
+    ("prefill", "w2"): 1_816_780_800 + 509_199_360,
+    ("decode", "fused_ffn"): 509_765_888 + 3_596_032,
+    ("skewed_decode", "fused_ffn"): 1_938_956_032 + 6_945_536,
+    ("decode+e4m3", "fused_ffn"): 256_420_864 + 3_050_240,
+    ("skewed_decode+e4m3", "fused_ffn"): 1_075_254_016 + 8_005_120,
+    ("routing_stress", "route"): 67_145_216 + 355_328,
 }
 
 # Records added to the default line (workload name, expert weight format).
