@@ -168,7 +168,7 @@ struct F8Cfg {
     static constexpr int kABytes = 2 * kBoxBytes;
     static constexpr int kBBytes = 2 * NT * 2 * kBK;  // 2 NT rows x 128 codes
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kScaleBytes = kGatherWarps * NT * 4;
+    static constexpr int kScaleBytes = kGatherWarps * NT * 4 + 64 * 4;  // + the x maxima
     static constexpr int kFixed = 1024 + C::kStagingBytes + C::kAuxBytes + kFusedReserve + kScaleBytes;
     static constexpr int kStagesRaw = (C::kMaxSmem - kFixed) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
@@ -545,6 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* tab_seq = reinterpret_cast<int*>(unit_tab + 2 * kUnitTable);
     RouteSmem* rs = reinterpret_cast<RouteSmem*>(tab_seq + kUnitTable);
     float* cscale = reinterpret_cast<float*>(rs + 1);  // F8: [gather warps][NT] row scales
+    uint32_t* xtab = reinterpret_cast<uint32_t*>(cscale + kGatherWarps * NT);  // F8: [T] max|x|
     // the routing scratch may run on into the epilogue staging that follows the ring
     static_assert(kRouteScratchBytes <= kRingBytes + C::kStagingBytes &&
                       kThreads / 32 * kMaxExperts * 4 <= kStagedLogitBytes && kThreads / 32 <= 20,
@@ -871,10 +872,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int g = (warp - 2) / W, wi = (warp - 2) % W;
             int* my_off = tok_off + (warp - 2) * NT;   // w13: element offset of each x row
             float* my_sc = cscale + (warp - 2) * NT;   // 2^s of each row
+            // x and act rows are re-read by every feature block's unit: keep them in
+            // L2 while the weight stream (evict-first) passes through
+            const uint64_t keep = l2_policy_evict_last();
             int q = 0;  // global stage sequence number (same as the producer's)
             int cur_tile = -1, cur_ph = -1, ready_tile = -1;
             bool ok = true;
             bool counters = false;
+            bool have_x = false;  // xtab filled (at the first w13 tile)
             for (int i = 0; ok; ++i) {
                 const Unit un = get(i);
                 if (__any_sync(0xffffffffu, un.ph >= kUnitEnd)) break;
@@ -895,6 +900,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ready_tile = un.tile;
                 }
+                if (un.ph == 0 && !have_x) {
+                    // every token's published max|x|, all at once, into a table in
+                    // shared memory (each gather warp writes the same values, and
+                    // reads only after its own writes)
+                    bool got = true;
+                    for (int tk = lane; tk < a.T; tk += 32) {
+                        uint32_t m = 0;
+                        got = token_xmax(a, tk, abort_flag, m) && got;
+                        xtab[tk] = m;
+                    }
+                    if (__any_sync(0xffffffffu, !got)) {
+                        if (lane == 0) flag_error(a.err, aux);
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    have_x = true;
+                }
                 if (un.tile != cur_tile || un.ph != cur_ph) {
                     __syncwarp();  // the previous tile's rows are all converted
                     bool got = true;
@@ -903,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (un.ph == 0) {
                             const int tok = rs->rows[t.row_start + j] / a.k;
                             my_off[j] = tok * a.H;
-                            got = token_xmax(a, tok, abort_flag, m) && got;
+                            m = xtab[tok];
                         } else {
                             m = (uint32_t)ld_acquire_gpu(
                                 reinterpret_cast<const int*>(a.act_max) + t.row_start + j);
@@ -950,8 +973,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               a.act + ((size_t)(kt + (c >> 2)) * a.R + t.row_start + j) *
                                                           kBK +
                                               (c & 3) * 16);
-                                v[u][0] = __ldcg(src);
-                                v[u][1] = __ldcg(src + 1);
+                                v[u][0] = ldcg_hint_v4(src, keep);
+                                v[u][1] = ldcg_hint_v4(src + 1, keep);
                             }
                         }
 #pragma unroll
@@ -1069,10 +1092,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // call's generation with release
             const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..255
             uint32_t* red = reinterpret_cast<uint32_t*>(staging);
+            const uint64_t keep = l2_policy_evict_last();  // the gather re-reads x from L2
             for (int tk = blockIdx.x; tk < a.T; tk += gridDim.x) {
                 const uint4* row = reinterpret_cast<const uint4*>(a.x + (size_t)tk * a.H);
                 uint32_t m2 = 0;
-                for (int i = et; i < a.H / 8; i += 256) m2 = absmax8(m2, __ldcg(row + i));
+                for (int i = et; i < a.H / 8; i += 256) m2 = absmax8(m2, ldcg_hint_v4(row + i, keep));
                 const uint32_t m = __reduce_max_sync(0xffffffffu, max(m2 & 0xffffu, m2 >> 16) << 16);
                 if (lane == 0) red[warp - kEpiWarp0] = m;
                 named_bar_sync(3, 256);

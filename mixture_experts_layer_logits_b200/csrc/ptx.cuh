@@ -192,6 +192,16 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last()
     return p;
 }
 
+// 16-byte global load cached in L2 only (as __ldcg), with an L2 cache policy.
+__device__ __forceinline__ uint4 ldcg_hint_v4(const void* p, uint64_t policy)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
+}
+
 // ---------------------------------------------------------------- cp.async (16 B)
 
 // 16-byte global -> shared copy (cp.async.cg: L2 only), with an L2 cache policy
