@@ -181,7 +181,6 @@ struct F8Cfg {
     static constexpr uint32_t kTxBytes = kABytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kSmemBytes = kFixed + kRingBytes;
-    static constexpr int kPf = 2;  // pair stages the producer prefetches into L2 ahead
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static_assert(kStages >= 3 && kStages <= kBarSlots, "pipeline depth");
     static_assert(kSmemBytes <= C::kMaxSmem, "shared memory");
@@ -714,7 +713,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr int kBox1 = F8 ? kBM * 2 * kBK : kATileBytes;  // second box
             constexpr int kKtStep = F8 ? 2 : 1;  // K tiles per ring stage
             constexpr uint32_t kTx = F8 ? F8C::kTxBytes : C::kTxBytes;
-            constexpr int kPf = F8C::kPf;
             uint8_t* const pring = ring;
             int stage = 0;
             uint32_t phase = 0;
@@ -751,15 +749,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int row0 = un.ph ? t.expert * a.H + un.fb * 2 * kBM
                                        : t.expert * 2 * a.I + un.fb * kBM;
                 const int row1 = un.ph ? row0 + kBM : row0 + a.I;
-                if constexpr (F8) {
-                    // the E4M3 ring holds fewer K tiles than the bf16 one: pair
-                    // stages kPf ahead of the TMA go to L2 now, to keep more weight
-                    // bytes in flight
-                    for (int kt = un.kt0 + 2; kt < min(un.kt1, un.kt0 + 2 * kPf); kt += 2) {
-                        tma_prefetch_l2_2d(tm, kt * kBK, row0);
-                        tma_prefetch_l2_2d(tm, kt * kBK, row1);
-                    }
-                }
                 for (int kt = un.kt0; kt < un.kt1; kt += kKtStep) {
                     if (!mbar_wait(&aux->empty[stage], phase ^ 1u, abort_flag)) {
                         flag_error(a.err, aux);
@@ -770,10 +759,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&aux->full[stage], kTx);
                     tma_load_2d(st, tm, &aux->full[stage], kt * kBK, row0, pol);
                     tma_load_2d(st + kBox1, tm, &aux->full[stage], kt * kBK, row1, pol);
-                    if (F8 && kt + 2 * kPf < un.kt1) {
-                        tma_prefetch_l2_2d(tm, (kt + 2 * kPf) * kBK, row0);
-                        tma_prefetch_l2_2d(tm, (kt + 2 * kPf) * kBK, row1);
-                    }
                     ++fills;
                     if (++stage == NS) {
                         stage = 0;
