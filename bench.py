@@ -54,8 +54,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (workload, kernel).  An entry is removed when its kernel changes, until it is
 # captured again.
 NCU_TRAFFIC = {
-    ("prefill", "w13"): 3_711_779_328 + 205_911_296,
-    ("prefill", "w2"): 1_816_780_800 + 509_199_360,
+    ("prefill", "w13"): 3_667_063_040 + 205_387_776,
+    ("prefill", "w2"): 1_828_432_128 + 510_838_272,
     ("decode", "fused_ffn"): 509_765_888 + 3_596_032,
     ("skewed_decode", "fused_ffn"): 1_938_956_032 + 6_945_536,
     ("decode+e4m3", "fused_ffn"): 255_764_992 + 3_243_008,

@@ -24,7 +24,6 @@ constexpr int kUmmaK = 16;      // K per tcgen05.mma (bf16)
 constexpr int kThreads = 512;   // 16 warps, roles below
 constexpr int kGatherWarps = 6;  // warps 2..7
 constexpr int kEpiWarp0 = 8;     // warps 8..15: two epilogue groups of four
-constexpr int kPrefetch = 4;     // weight K-tiles brought to L2 ahead of their TMA
 constexpr int kStageRows = 8;    // token rows per epilogue staging buffer
 constexpr int kStageRowBytes = 512;  // one token row: 256 bf16 outputs
 constexpr int kATileBytes = kBM * kBK * 2;

@@ -288,16 +288,6 @@ __global__ void __launch_bounds__(GCfg<MODE, NT>::kThreads, 1)
                         tma_load_2d_nohint(st + 2 * kATileBytes, &tm_act, &aux->full[stage],
                                            kt * kBK, t.row_start);
                     }
-                    // weight tiles kPrefetch stages ahead go to L2 now, so the TMA that
-                    // needs them later finds them there (the ring holds only a few stages)
-                    // (weight-streaming shapes read each block once: nothing to gain there)
-                    if (!a.weights_evict_first && kt + kPrefetch < kt1) {
-                        const int row = MODE == 0 ? t.expert * 2 * a.I + fb * kBM
-                                                  : t.expert * a.H + fb * 2 * kBM;
-                        const int row1 = MODE == 0 ? row + a.I : row + kBM;
-                        tma_prefetch_l2_2d(&tm_w, (kt + kPrefetch) * kBK, row);
-                        tma_prefetch_l2_2d(&tm_w, (kt + kPrefetch) * kBK, row1);
-                    }
                     ++fills;
                     if (++stage == C::kStages) {
                         stage = 0;

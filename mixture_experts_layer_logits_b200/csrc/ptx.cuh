@@ -152,15 +152,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
         : "memory");
 }
 
-// Bring a 2D tile into L2 only (no shared memory, no completion tracking).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int c0, int c1)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
-}
-
 // Same, without an L2 cache policy.
 __device__ __forceinline__ void tma_load_2d_nohint(void* dst, const void* tmap, uint64_t* bar,
                                                    int c0, int c1)
