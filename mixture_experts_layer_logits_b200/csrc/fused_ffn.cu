@@ -160,7 +160,7 @@ using FCfg = Cfg<0, NT, kFusedReserve>;
 // warps.  Tensor memory: kNBuf accumulators of 4 NT columns, box 0 (gate block,
 // or the first w2 row block) at column 0 (hi terms in [0, n), lo in [n, 2n)),
 // box 1 at column 2 NT.  After the routing tables, one fp32 row scale per row
-// of the tile for each gather warp.
+// of the tile for each gather warp, then the T token maxima (64 words).
 template <int NT>
 struct F8Cfg {
     using C = FCfg<NT>;
