@@ -52,3 +52,27 @@ def test_stage_work_counts_e4m3_weights_at_one_byte_plus_row_scales():
     assert f8["fused_ffn"]["bytes"] == n * (3 * I * H + (2 * I + H) * 4) + rest
     assert f8["fused_ffn"]["flops"] == bf["fused_ffn"]["flops"]  # same bf16 products
     assert f8["route_permute"] == bf["route_permute"] and f8["combine"] == bf["combine"]
+
+
+def test_traffic_table_keys_name_real_workloads_and_stages():
+    """Every measured DRAM-bytes entry is keyed by a workload the bench knows (with
+    "+e4m3" for E4M3 weights) and a stage its roofline can pick, and the
+    dominant kernel of every suite record but the tiny layer has one."""
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_logits_b200 import workloads as wl
+
+    stages = set(bench.stage_work(wl.WORKLOADS["decode"], 1)) | {"route"}
+    for (tag, stage), traffic in bench.NCU_TRAFFIC.items():
+        name, _, fmt = tag.partition("+")
+        assert name in wl.WORKLOADS and fmt in ("", "e4m3"), tag
+        assert stage in stages, stage
+        assert isinstance(traffic, int) and traffic > 0
+    for name, fmt in [("prefill", "bf16")] + bench.SUITE:
+        if name == "tiny":
+            continue
+        stage = {"prefill": "w13", "routing_stress": "route"}.get(name, "fused_ffn")
+        tag = name + ("+e4m3" if fmt == "e4m3" else "")
+        assert (tag, stage) in bench.NCU_TRAFFIC, (tag, stage)
