@@ -58,8 +58,8 @@ NCU_TRAFFIC = {
     ("prefill", "w2"): 1_828_432_128 + 510_838_272,
     ("decode", "fused_ffn"): 509_765_888 + 3_596_032,
     ("skewed_decode", "fused_ffn"): 1_938_956_032 + 6_945_536,
-    ("decode+e4m3", "fused_ffn"): 255_764_992 + 3_243_008,
-    ("skewed_decode+e4m3", "fused_ffn"): 971_161_344 + 7_240_960,
+    ("decode+e4m3", "fused_ffn"): 255_728_384 + 3_075_840,
+    ("skewed_decode+e4m3", "fused_ffn"): 971_040_768 + 7_290_368,
     ("routing_stress", "route"): 67_145_216 + 355_328,
 }
 
