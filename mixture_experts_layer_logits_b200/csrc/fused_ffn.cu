@@ -605,7 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // slice adds epilogue publishes and combine reads (same-B200 A/B: 16 waves
     // 101.4 us decode / 360.7 us skewed decode, 4 waves 98.2 / 341.8).  E4M3
     // units stream half the bytes, so ~2 waves (decode with E4M3 weights: 4 waves
-    // 68.9 us, 2 waves 66.5 us, 1 wave 66.4 us; skewed decode unchanged).
+    // 68.9 us, 2 waves 66.5 us, 1 wave 66.4 us; skewed decode unchanged); bf16 units
+    // keep 4 (2 waves: decode 100.6 -> 101.8 us).
     const int s2w = split_count(ntiles * a.fb2, a.s2_max, a.kt2, a.min_kt_per_split, F8 ? 2 : 4);
     int ktps2 = (a.kt2 + s2w - 1) / s2w;
     if (F8) ktps2 = (ktps2 + 1) & ~1;  // whole pair stages
